@@ -1,0 +1,180 @@
+"""CPU oracle for the FP8 block-scaled linear — TEST INFRASTRUCTURE ONLY.
+
+A ctypes wrapper around ``fp8q_oracle.c``: the plain, slow CPU restatement of
+per-token-group FP8 activation quantization, 128x128 block weight
+quantization and the float64 dequantized GEMM reference (pages
+"spark_model/layers/ops/dispatch_proj.rs" and
+"spark_model/layers/ops/fp8_act_quant_floor.rs").
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. The product library never does, and
+this package never imports the product.
+
+Every function takes and returns numpy arrays. bf16 values travel as their
+uint16 bit patterns and e4m3 values as uint8 codes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fp8q_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+GROUP = 128
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with plain IEEE arithmetic (no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+               "-fno-fast-math", "-o", _LIB + ".tmp", _SRC, "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        U32 = ctypes.c_uint32
+        lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.oracle_bf16_to_f32.restype = ctypes.c_float
+        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_decode.restype = ctypes.c_double
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_e4m3_encode_array.argtypes = [P, ctypes.c_size_t, P]
+        lib.oracle_e4m3_encode_array.restype = None
+        lib.oracle_m_pad.argtypes = [U32]
+        lib.oracle_m_pad.restype = U32
+        lib.oracle_quant_act.argtypes = [P, U32, U32, P, P, P]
+        lib.oracle_quant_act.restype = ctypes.c_int
+        lib.oracle_quant_weight.argtypes = [P, U32, U32, P, P]
+        lib.oracle_quant_weight.restype = ctypes.c_int
+        lib.oracle_gemm_ref_rows.argtypes = [P, P, P, P, U32, U32, P, ctypes.c_size_t,
+                                             ctypes.c_size_t, P]
+        lib.oracle_gemm_ref_rows.restype = None
+        lib.oracle_check_tolerance.argtypes = [P, P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_double)]
+        lib.oracle_check_tolerance.restype = ctypes.c_size_t
+        _lib = lib
+        return lib
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def bf16_to_f32(h: int) -> float:
+    return float(_load().oracle_bf16_to_f32(int(h)))
+
+
+def e4m3_decode(code: int) -> float:
+    return float(_load().oracle_e4m3_decode(int(code)))
+
+
+def e4m3_encode(t: float) -> int:
+    return int(_load().oracle_e4m3_encode(float(t)))
+
+
+def e4m3_encode_array(t: np.ndarray) -> np.ndarray:
+    """Encode each fp32 value with the scalar encoder (for sweeps)."""
+    t = np.ascontiguousarray(t, dtype=np.float32).ravel()
+    out = np.empty(t.size, np.uint8)
+    _load().oracle_e4m3_encode_array(_ptr(t), t.size, _ptr(out))
+    return out
+
+
+def m_pad(m: int) -> int:
+    return int(_load().oracle_m_pad(int(m)))
+
+
+def quant_act(x_bf16: np.ndarray):
+    """bf16 bits [M,K] -> (q [M,K] u8, s_row [M,K/128] f32, s_kmajor [K/128, ceil16(M)] f32)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    m, k = x.shape
+    if k % GROUP:
+        raise ValueError("k must be a multiple of 128")
+    g = k // GROUP
+    q = np.empty((m, k), np.uint8)
+    s_row = np.empty((m, g), np.float32)
+    s_k = np.empty((g, m_pad(m)), np.float32)
+    rc = _load().oracle_quant_act(_ptr(x), m, k, _ptr(q), _ptr(s_row), _ptr(s_k))
+    assert rc == 0
+    return q, s_row, s_k
+
+
+def quant_weight(w_bf16: np.ndarray):
+    """bf16 bits [N,K] -> (wq [N,K] u8, w_scale [N/128, K/128] f32)."""
+    w = np.ascontiguousarray(w_bf16, dtype=np.uint16)
+    n, k = w.shape
+    if n % GROUP or k % GROUP:
+        raise ValueError("n and k must be multiples of 128")
+    wq = np.empty((n, k), np.uint8)
+    ws = np.empty((n // GROUP, k // GROUP), np.float32)
+    rc = _load().oracle_quant_weight(_ptr(w), n, k, _ptr(wq), _ptr(ws))
+    assert rc == 0
+    return wq, ws
+
+
+def gemm_ref(q: np.ndarray, a_scale_row: np.ndarray, wq: np.ndarray, w_scale: np.ndarray,
+             rows: np.ndarray | None = None, threads: int = 1) -> np.ndarray:
+    """Float64 reference Y[rows, N] of the block-scaled GEMM.
+
+    ``a_scale_row`` is the row-major [M, K/128] activation scale. ``rows``
+    selects output rows (default: all). ``threads`` > 1 splits the rows over
+    Python threads; the C loop itself is unchanged.
+    """
+    lib = _load()
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    a_s = np.ascontiguousarray(a_scale_row, dtype=np.float32)
+    wq = np.ascontiguousarray(wq, dtype=np.uint8)
+    ws = np.ascontiguousarray(w_scale, dtype=np.float32)
+    m, k = q.shape
+    n = wq.shape[0]
+    assert wq.shape[1] == k and a_s.shape == (m, k // GROUP) and ws.shape == (n // GROUP, k // GROUP)
+    if rows is None:
+        rows_arr = np.arange(m, dtype=np.int64)
+    else:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        assert rows_arr.size == 0 or (rows_arr.min() >= 0 and rows_arr.max() < m)
+    cnt = rows_arr.size
+    ref = np.empty((cnt, n), np.float64)
+    args = (_ptr(q), _ptr(a_s), _ptr(wq), _ptr(ws), n, k, _ptr(rows_arr))
+    if threads <= 1 or cnt <= 1:
+        lib.oracle_gemm_ref_rows(*args, 0, cnt, _ptr(ref))
+    else:
+        bounds = np.linspace(0, cnt, min(threads, cnt) + 1).astype(int)
+        with ThreadPoolExecutor(len(bounds) - 1) as ex:
+            futs = [ex.submit(lib.oracle_gemm_ref_rows, *args, int(a), int(b - a), _ptr(ref))
+                    for a, b in zip(bounds[:-1], bounds[1:])]
+            for f in futs:
+                f.result()
+    return ref
+
+
+def check_tolerance(y_bf16: np.ndarray, ref: np.ndarray):
+    """Return (number of failing elements, worst err/bound ratio) for
+    |y-ref| <= 8e-3|ref| + 1e-3 rms(ref)."""
+    y = np.ascontiguousarray(y_bf16, dtype=np.uint16).ravel()
+    r = np.ascontiguousarray(ref, dtype=np.float64).ravel()
+    assert y.size == r.size
+    worst = ctypes.c_double(0.0)
+    bad = _load().oracle_check_tolerance(_ptr(y), _ptr(r), y.size, ctypes.byref(worst))
+    return int(bad), float(worst.value)

@@ -1,0 +1,316 @@
+/*
+ * fp8q oracle — TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, obviously correct CPU restatement of the W8A8 FP8
+ * block-scaled linear projection described on the pages
+ * "spark_model/layers/ops/dispatch_proj.rs" (doc comments of
+ * `cublas_fp8_proj`, `cublas_fp8_proj_prequant`, `fp8_act_scale_to_kmajor`,
+ * `cublas_fp8_m_pad`, `dequant_fp8_bf16_into`) and
+ * "spark_model/layers/ops/fp8_act_quant_floor.rs" (module header).
+ *
+ * Only the test suite, the smoke check and the benchmark's CPU-baseline leg
+ * may load this library. The product path (libfp8q.so) never links, loads or
+ * calls it, and the two share no code, header, table or helper.
+ *
+ * The pages name the activation quantizer (`per_token_group_quant_fp8`,
+ * "FP8 + per-[token,128-of-K] scales", "FP32 activation scales", "FP8 E4M3")
+ * but never print its body. The arithmetic here is the method's standard
+ * definition, written out step by step:
+ *   amax  = max_j |x_j|                       over one 128-wide K group
+ *   s     = max(amax, 1e-10f) / 448.0f        one IEEE fp32 division
+ *   q_j   = e4m3_rne_satfinite(x_j / s)       IEEE fp32 division, then
+ *                                             round-to-nearest-even into
+ *                                             OCP E4M3FN, saturating at 448
+ * Precision: the scale and the quotients are fp32 (the pages fix FP32
+ * scales); the code decision is taken on that fp32 quotient. The encoder
+ * works in double, where every step below is exact.
+ *
+ * Build: gcc -O2 -std=c11 -fPIC -shared (no -ffast-math, no -ffp-contract
+ * beyond "off": fp32 results must be IEEE single-rounded).
+ */
+#include <float.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#if !defined(FLT_EVAL_METHOD) || FLT_EVAL_METHOD != 0
+#error "the oracle needs fp32 expressions evaluated in fp32 (FLT_EVAL_METHOD == 0)"
+#endif
+
+#define GROUP 128            /* K-group width and weight block edge */
+#define E4M3_MAX 448.0       /* largest finite OCP E4M3FN magnitude */
+
+/* ---------------------------------------------------------------- bf16 -- */
+
+/* bf16 is the top half of an IEEE binary32: widening is a 16-bit shift. */
+float oracle_bf16_to_f32(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* ---------------------------------------------------------------- e4m3 -- */
+
+/*
+ * Decode one OCP E4M3FN code ("FP8 E4M3", dispatch_proj.rs,
+ * `dequant_fp8_bf16_into` doc: every such value is exactly a bf16).
+ * Layout: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits.
+ * Exponent field 0 holds subnormals m/8 * 2^-6. The only NaNs are
+ * S.1111.111; there is no infinity.
+ */
+double oracle_e4m3_decode(uint8_t code)
+{
+    int sign = (code >> 7) & 1;
+    int e = (code >> 3) & 0xF;
+    int m = code & 0x7;
+    double mag;
+    if (e == 0xF && m == 0x7)
+        return NAN;
+    if (e == 0)
+        mag = ldexp((double)m / 8.0, -6);
+    else
+        mag = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -mag : mag;
+}
+
+/* Round a non-negative double to the nearest integer, ties to even. */
+static double round_half_even(double v)
+{
+    double f = floor(v);
+    double frac = v - f; /* exact for the values used here */
+    if (frac > 0.5)
+        return f + 1.0;
+    if (frac < 0.5)
+        return f;
+    return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;
+}
+
+/*
+ * Encode one finite fp32 value into E4M3FN with round-to-nearest-even and
+ * saturation to the largest finite value (448), keeping the sign of zero.
+ *   |t| >= 448           -> 0x7E | sign (values in (448,464) round to 448
+ *                           anyway; larger ones would round to 480, which the
+ *                           format cannot hold, so saturation clamps them)
+ *   |t| <  2^-6          -> subnormal: mantissa = RNE(|t| / 2^-9); a result
+ *                           of 8 is the smallest normal, code 0x08
+ *   otherwise            -> e = floor(log2 |t|), mantissa = RNE((|t|/2^e - 1)*8);
+ *                           a mantissa of 8 carries into the exponent
+ */
+uint8_t oracle_e4m3_encode(float t)
+{
+    uint8_t sign = signbit(t) ? 0x80 : 0x00;
+    double a = fabs((double)t);
+    int e;
+    double r;
+    if (a >= E4M3_MAX)
+        return (uint8_t)(sign | 0x7E);
+    if (a < ldexp(1.0, -6)) {
+        r = round_half_even(a * 512.0); /* a / 2^-9, exact */
+        return (uint8_t)(sign | (uint8_t)r); /* r in 0..8; 8 == code 0x08 */
+    }
+    e = (int)floor(log2(a));
+    /* log2 of a double can be off by one ulp near powers of two: fix e so
+       that 2^e <= a < 2^(e+1) holds exactly. */
+    while (ldexp(1.0, e) > a)
+        e--;
+    while (ldexp(1.0, e + 1) <= a)
+        e++;
+    r = round_half_even((ldexp(a, -e) - 1.0) * 8.0);
+    if (r == 8.0) {
+        r = 0.0;
+        e += 1;
+    }
+    return (uint8_t)(sign | (uint8_t)(((e + 7) << 3) | (int)r));
+}
+
+/* ------------------------------------------------- group quantization -- */
+
+/*
+ * Quantize one group of `len` values (given as fp32, each exactly a bf16)
+ * with the shared scale: steps a1 (amax), a2 (scale) and a3 (codes).
+ * Returns the fp32 scale.
+ */
+static float quantize_group(const float *x, size_t stride, size_t len, uint8_t *q, size_t qstride)
+{
+    float amax = 0.0f;
+    float s;
+    size_t j;
+    for (j = 0; j < len; j++) {
+        float v = fabsf(x[j * stride]);
+        if (v > amax)
+            amax = v;
+    }
+    s = (amax > 1e-10f ? amax : 1e-10f) / 448.0f; /* one fp32 division */
+    for (j = 0; j < len; j++) {
+        float t = x[j * stride] / s;              /* one fp32 division */
+        q[j * qstride] = oracle_e4m3_encode(t);
+    }
+    return s;
+}
+
+/* ceil16(M): the padded token extent of the K-major scales
+   (dispatch_proj.rs, `cublas_fp8_m_pad`). */
+uint32_t oracle_m_pad(uint32_t m)
+{
+    return (m + 15u) / 16u * 16u;
+}
+
+/*
+ * Per-token, per-128-K-group activation quantization with both scale
+ * layouts (dispatch_proj.rs: `cublas_fp8_proj` quantizes "the real M
+ * tokens"; `fp8_act_scale_to_kmajor` rewrites `[M, K/128]` into
+ * `[K/128, M_pad]` and zero-fills rows M..M_pad).
+ *   x        bf16 bits, [m, k] row-major
+ *   q        e4m3 codes, [m, k] row-major
+ *   s_row    fp32, [m, k/128] row-major            (may be NULL)
+ *   s_kmaj   fp32, [k/128, ceil16(m)]; s_kmaj[g][t] = s_row[t][g] for t < m,
+ *            +0.0f for m <= t < ceil16(m)          (may be NULL)
+ * Returns 0, or -1 if k is not a multiple of 128.
+ */
+int oracle_quant_act(const uint16_t *x, uint32_t m, uint32_t k,
+                     uint8_t *q, float *s_row, float *s_kmaj)
+{
+    uint32_t G, mp, t, g, j;
+    float buf[GROUP];
+    if (k % GROUP != 0)
+        return -1;
+    G = k / GROUP;
+    mp = oracle_m_pad(m);
+    for (t = 0; t < m; t++) {
+        for (g = 0; g < G; g++) {
+            const uint16_t *xg = x + (size_t)t * k + (size_t)g * GROUP;
+            float s;
+            for (j = 0; j < GROUP; j++)
+                buf[j] = oracle_bf16_to_f32(xg[j]);
+            s = quantize_group(buf, 1, GROUP, q + (size_t)t * k + (size_t)g * GROUP, 1);
+            if (s_row)
+                s_row[(size_t)t * G + g] = s;
+            if (s_kmaj)
+                s_kmaj[(size_t)g * mp + t] = s;
+        }
+    }
+    if (s_kmaj)
+        for (g = 0; g < G; g++)
+            for (t = m; t < mp; t++)
+                s_kmaj[(size_t)g * mp + t] = 0.0f;
+    return 0;
+}
+
+/*
+ * Weight pre-quantization per 128x128 block: the same amax / scale / code
+ * steps taken over a whole block. Layout follows the block-scaled
+ * `Fp8Weight` of dispatch_proj.rs (`dequant_fp8_bf16_into` doc):
+ *   w        bf16 bits [n, k] row-major
+ *   wq       e4m3 codes [n, k] row-major
+ *   w_scale  fp32 [n/128, k/128] row-major, read as scale[(r/128)*(k/128) + c/128]
+ * Returns 0, or -1 unless n and k are multiples of 128.
+ */
+int oracle_quant_weight(const uint16_t *w, uint32_t n, uint32_t k,
+                        uint8_t *wq, float *w_scale)
+{
+    uint32_t NB, G, bn, bg, r, c;
+    float blk[GROUP * GROUP];
+    uint8_t qb[GROUP * GROUP];
+    if (n % GROUP != 0 || k % GROUP != 0)
+        return -1;
+    NB = n / GROUP;
+    G = k / GROUP;
+    for (bn = 0; bn < NB; bn++) {
+        for (bg = 0; bg < G; bg++) {
+            float s;
+            for (r = 0; r < GROUP; r++)
+                for (c = 0; c < GROUP; c++)
+                    blk[r * GROUP + c] = oracle_bf16_to_f32(
+                        w[(size_t)(bn * GROUP + r) * k + (size_t)bg * GROUP + c]);
+            s = quantize_group(blk, 1, (size_t)GROUP * GROUP, qb, 1);
+            w_scale[(size_t)bn * G + bg] = s;
+            for (r = 0; r < GROUP; r++)
+                for (c = 0; c < GROUP; c++)
+                    wq[(size_t)(bn * GROUP + r) * k + (size_t)bg * GROUP + c] = qb[r * GROUP + c];
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------- GEMM reference -- */
+
+/*
+ * Float64 dequantized reference of the block-scaled GEMM
+ * (dispatch_proj.rs, `cublas_fp8_proj` / `cublas_fp8_proj_prequant`:
+ * out[M,N] = act[M,K] @ weight^T, activation scales per [token, 128 of K],
+ * weight scales per 128x128 block):
+ *   ref[i][col] = sum_k  deq(q[r_i][k]) * a_s[r_i][k/128]
+ *                      * deq(wq[col][k]) * w_s[col/128][k/128]
+ * for each requested row r_i (rows == NULL means rows 0..n_rows-1).
+ *   q      e4m3 [m, k];  a_s  fp32 [m, k/128] row-major (the definition's
+ *          own indexing; the K-major copy is a layout of the same numbers)
+ *   wq     e4m3 [n, k];  w_s  fp32 [n/128, k/128]
+ *   ref    float64 [n_rows, n]
+ * Rows are independent; `first`/`count` select a slice of the requested
+ * rows so a caller may split the work over threads.
+ */
+void oracle_gemm_ref_rows(const uint8_t *q, const float *a_s,
+                          const uint8_t *wq, const float *w_s,
+                          uint32_t n, uint32_t k,
+                          const int64_t *rows, size_t first, size_t count,
+                          double *ref)
+{
+    double lut[256];
+    uint32_t G = k / GROUP;
+    size_t i;
+    uint32_t col, kk;
+    for (i = 0; i < 256; i++)
+        lut[i] = oracle_e4m3_decode((uint8_t)i);
+    for (i = first; i < first + count; i++) {
+        int64_t r = rows ? rows[i] : (int64_t)i;
+        const uint8_t *qa = q + (size_t)r * k;
+        const float *sa = a_s + (size_t)r * G;
+        for (col = 0; col < n; col++) {
+            const uint8_t *qw = wq + (size_t)col * k;
+            const float *sw = w_s + (size_t)(col / GROUP) * G;
+            double acc = 0.0;
+            for (kk = 0; kk < k; kk++)
+                acc += lut[qa[kk]] * (double)sa[kk / GROUP] * lut[qw[kk]] * (double)sw[kk / GROUP];
+            ref[i * n + col] = acc;
+        }
+    }
+}
+
+/*
+ * The acceptance test of a computed output against the reference:
+ *   |y - ref| <= 8e-3 * |ref| + 1e-3 * rms(ref)   for every element,
+ * rms taken over all `count` reference values given. `y` is bf16 bits.
+ * Returns the number of elements that fail; writes the worst ratio
+ * |y-ref| / (8e-3|ref| + 1e-3 rms) to *worst.
+ */
+size_t oracle_check_tolerance(const uint16_t *y, const double *ref, size_t count, double *worst)
+{
+    double ss = 0.0, rms, w = 0.0;
+    size_t i, bad = 0;
+    for (i = 0; i < count; i++)
+        ss += ref[i] * ref[i];
+    rms = count ? sqrt(ss / (double)count) : 0.0;
+    for (i = 0; i < count; i++) {
+        double yv = (double)oracle_bf16_to_f32(y[i]);
+        double err = fabs(yv - ref[i]);
+        double bound = 8e-3 * fabs(ref[i]) + 1e-3 * rms;
+        double ratio = bound > 0.0 ? err / bound : (err > 0.0 ? INFINITY : 0.0);
+        if (!(err <= bound))
+            bad++;
+        if (ratio > w || ratio != ratio)
+            w = ratio;
+    }
+    if (worst)
+        *worst = w;
+    return bad;
+}
+
+/* Encode `count` fp32 values one by one with oracle_e4m3_encode (sweeps). */
+void oracle_e4m3_encode_array(const float *t, size_t count, uint8_t *out)
+{
+    size_t i;
+    for (i = 0; i < count; i++)
+        out[i] = oracle_e4m3_encode(t[i]);
+}
