@@ -1,0 +1,409 @@
+#!/usr/bin/env python
+"""Benchmark of the W8A8 FP8 block-scaled linear on B200.
+
+One step = one fused linear call (fp8q_linear: per-token-group FP8
+quantization of X plus the block-scaled FP8 GEMM) on one batch of
+synthetic activations, at the prefill projection M=1168, K=5120, N=17408
+(the up-projection shape the pages quote for act-quant GB/s and linear
+TFLOP/s). Inputs are resident in HBM when the timed region starts; the
+steps rotate over three input sets (X, W, Y and workspace, ~450 MB) so
+no step reads what the previous one left in the 126 MB L2.
+
+Prints ONE JSON line (rank 0). With --gpus N under torchrun each rank runs
+its own replica on its own tokens (weak scaling; the path has no exchange
+step), and the time is the max over ranks.
+
+--impl reference times the CPU oracle (the plain restatement of the method
+in oracle/) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "FP8 block-scaled linear TFLOP/s & act-quant GB/s, % of B200 roofline"
+WORKLOADS = {
+    "prefill_m1168_n17408_k5120": dict(m=1168, n=17408, k=5120, p=0.01, sigma=20.0, number=4),
+    "prefill_m4576_n6144_k6144": dict(m=4576, n=6144, k=6144, p=0.001, sigma=50.0, number=5),
+    "prefill_m4576_n6144_k17408": dict(m=4576, n=6144, k=17408, p=0.001, sigma=50.0, number=5),
+    "decode_m25_n6144_k5120": dict(m=25, n=6144, k=5120, p=0.01, sigma=20.0, number=2),
+    "decode_m25_n5120_k17408": dict(m=25, n=5120, k=17408, p=0.01, sigma=20.0, number=3),
+}
+DEFAULT_WORKLOAD = "prefill_m1168_n17408_k5120"
+N_SETS = 3
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def quant_bytes(m, k):
+    g = k // 128
+    mp = -(-m // 16) * 16
+    return 2 * m * k + m * k + 4 * g * mp  # read X, write Q and the K-major scales
+
+
+def gemm_hbm_bytes(m, n, k):
+    g = k // 128
+    mp = -(-m // 16) * 16
+    return m * k + n * k + 4 * g * mp + 4 * (n // 128) * g + 2 * m * n
+
+
+def read_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded from an ncu capture in profiles/traffic.txt,
+    or None when absent or when the kernel sources changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    from fp8_block_scaled_group_b200 import build as pkg_build
+    import hashlib
+    h = hashlib.sha256()
+    for src in pkg_build.sources():
+        with open(src, "rb") as f:
+            h.update(f.read())
+    digest = h.hexdigest()[:16]
+    with open(path) as f:
+        for line in f:
+            parts = line.split("#", 1)[0].split()
+            if len(parts) == 4 and parts[0] == kernel and parts[1] == workload and parts[3] == digest:
+                return float(parts[2])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            p = [x.strip() for x in ln.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                smax = float(p[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, p[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, world: int) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ CPU oracle --
+
+def cpu_oracle_sample(wl: dict, seed: int, target_s: float, threads: int):
+    """Time the oracle on a bounded sample of one step: quantize R rows of X and
+    compute those R rows of the float64 reference output. Returns
+    (TFLOP/s equivalent of 2*R*N*K / time, rows, seconds)."""
+    import oracle
+    from fp8_block_scaled_group_b200 import inputs
+    m, n, k = wl["m"], wl["n"], wl["k"]
+    xb = inputs.activations(m, k, seed, wl["p"], wl["sigma"])
+    wb = inputs.weights(n, k, wl["number"] + 1000)
+    wq, ws = oracle.quant_weight(wb)   # weight preparation is not part of the step
+
+    def run(rows):
+        t0 = time.perf_counter()
+        q, s_row, _ = oracle.quant_act(np.ascontiguousarray(xb[:rows]))
+        oracle.gemm_ref(q, s_row, wq, ws, threads=threads)
+        return time.perf_counter() - t0
+
+    r = min(m, max(threads, 1))
+    t = run(r)
+    rows = int(min(m, max(r, r * target_s / max(t, 1e-3))))
+    rows = max(threads, rows - rows % max(threads, 1)) if rows >= threads else rows
+    t = run(rows)
+    return 2.0 * rows * n * k / t / 1e12, rows, t
+
+
+def reference_arm(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = WORKLOADS[args.workload]
+    threads = os.cpu_count() or 1
+    per_step = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    rows = 0
+    for i in range(args.warmup + args.steps):
+        v, rows, _ = cpu_oracle_sample(wl, 1000 + wl["number"], per_step, threads)
+        if i >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals)
+    flops = 2.0 * wl["m"] * wl["n"] * wl["k"]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": flops / (value * 1e12) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "m": wl["m"], "n": wl["n"], "k": wl["k"]},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{rows} of {wl['m']} token rows per step (quantize + float64 GEMM rows), "
+                                   f"scaled to the metric's unit"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------- our arm --
+
+def ours_arm(args):
+    import torch
+    from fp8_block_scaled_group_b200 import api, inputs
+
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = WORKLOADS[args.workload]
+    m, n, k = wl["m"], wl["n"], wl["k"]
+    g = k // 128
+    seed_base = 1000 + wl["number"]
+
+    # Input sets: each rank draws its own tokens (weak scaling).
+    sets = []
+    for i in range(N_SETS):
+        xb = inputs.activations(m, k, seed_base + 7919 * (rank * N_SETS + i), wl["p"], wl["sigma"])
+        wb = inputs.weights(n, k, seed_base + i)
+        x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
+        w = torch.from_numpy(wb.view(np.int16)).view(torch.bfloat16).to(dev)
+        wq, ws = api.quant_weight(w)
+        del w
+        work = torch.empty(api.linear_workspace_bytes(m, k), dtype=torch.uint8, device=dev)
+        y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        sets.append(dict(x=x, wq=wq, ws=ws, work=work, y=y, xb=xb))
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        s = sets[i % N_SETS]
+        api.linear(s["x"], s["wq"], s["ws"], workspace=s["work"], out=s["y"])
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    launches0 = api.launch_count()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    launches = api.launch_count() - launches0
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
+
+    # Kernel breakdown over the same rotation: quantizer and GEMM launched
+    # separately with events around each on the launching stream.
+    q_ms, g_ms = [], []
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    for i in range(args.steps):
+        s = sets[i % N_SETS]
+        off = api.linear_scale_offset(m, k)
+        q = s["work"][:m * k].view(m, k)
+        s_k = s["work"][off:off + 4 * g * api.m_pad(m)].view(torch.float32).view(g, api.m_pad(m))
+        evs[0].record(stream)
+        api.quant_act(s["x"], out=(q, None, s_k))
+        evs[1].record(stream)
+        api.gemm_blockscaled(q, s_k, s["wq"], s["ws"], out=s["y"])
+        evs[2].record(stream)
+        torch.cuda.synchronize()
+        q_ms.append(evs[0].elapsed_time(evs[1]))
+        g_ms.append(evs[1].elapsed_time(evs[2]))
+    clk = clocks.stop()
+
+    # End to end through the public call with host buffers: pinned X in,
+    # fused linear, Y back to pinned host memory, every step.
+    x_host = [torch.from_numpy(s["xb"].view(np.int16)).view(torch.bfloat16).pin_memory() for s in sets]
+    y_host = torch.empty((m, n), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty((m, k), dtype=torch.bfloat16, device=dev)
+
+    def e2e_step(i):
+        s = sets[i % N_SETS]
+        x_dev.copy_(x_host[i % N_SETS], non_blocking=True)
+        api.linear(x_dev, s["wq"], s["ws"], workspace=s["work"], out=s["y"])
+        y_host.copy_(s["y"], non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+
+    flops = 2.0 * m * n * k
+    value = flops * world * args.steps / (ms_total * 1e-3) / 1e12
+    e2e_value = flops * world * args.steps / (e2e_ms * 1e-3) / 1e12
+    hbm, bf16, bf16_sus, src = load_peaks()
+    fp8_peak = bf16 * 2.0  # fp8 dense = 2x bf16 dense (nominal 4.5 / 2.25 PF)
+    gemm_us = statistics.mean(g_ms) * 1e3
+    quant_us = statistics.mean(q_ms) * 1e3
+    gemm_tf = flops / (gemm_us * 1e-6) / 1e12
+    quant_gbs = quant_bytes(m, k) / (quant_us * 1e-6) / 1e9
+    traffic = read_traffic("gemm_blockscaled_kernel", args.workload)
+    q_traffic = read_traffic("quant_act_multi_kernel", args.workload)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        v, rows, t = cpu_oracle_sample(wl, seed_base, args.cpu_seconds, threads)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{rows} of {m} token rows of one step (quantize + float64 GEMM rows), "
+                         f"{t:.1f} s, scaled to TFLOP/s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+            "config": {"workload": args.workload, "m": m, "n": n, "k": k, "parallelism": f"replicas{world}",
+                       "l2": f"{N_SETS} rotating input sets ({N_SETS * (m * k * 2 + n * k + m * n * 2) / 1e6:.0f} MB) > L2"},
+            "roofline": {"bound": "tensor", "kernel": "gemm_blockscaled_kernel", "achieved": gemm_tf,
+                         "peak": fp8_peak, "unit": "TFLOP/s", "frac": gemm_tf / fp8_peak, "traffic": traffic,
+                         "peak_source": f"{src} bf16 burst x 2 (fp8:bf16 nominal ratio)",
+                         "algorithmic_bytes": gemm_hbm_bytes(m, n, k), "us": gemm_us},
+            "act_quant": {"bound": "hbm", "kernel": "quant_act", "achieved": quant_gbs, "peak": hbm, "unit": "GB/s",
+                          "frac": quant_gbs / hbm, "us": quant_us, "bytes": quant_bytes(m, k), "traffic": q_traffic,
+                          "peak_source": f"{src} copy bandwidth"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": m * k * 2,
+                    "d2h_bytes_per_step": m * n * 2},
+            "gpu_launches": int(sum_over_ranks(launches, world)),
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    barrier(world)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    if args.impl == "reference":
+        return reference_arm(args)
+    return ours_arm(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,144 @@
+"""PyTorch-facing calls of the fp8q C ABI.
+
+Each function takes CUDA tensors, checks dtype/shape/contiguity, allocates
+outputs with torch when the caller gives none, and passes raw device
+pointers plus the current CUDA stream to libfp8q.so. No arithmetic of the
+method happens here.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+
+AUTO, SINGLE, MULTI = 0, 1, 2
+GROUP = 128
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _p(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, dtype, shape, name):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def m_pad(m: int) -> int:
+    return int(_lib.load().fp8q_m_pad(m))
+
+
+def quant_pick(m: int, k: int, sm_count: int, requested: int = AUTO) -> _lib.QuantPick:
+    out = _lib.QuantPick()
+    _lib.check(_lib.load().fp8q_quant_pick(m, k, sm_count, requested, ctypes.byref(out)), "fp8q_quant_pick")
+    return out
+
+
+def quant_floor_min_m(k: int, sm_count: int, groups_per_cta: int, rows_per_cta: int, min_ctas_per_sm: int) -> int:
+    return int(_lib.load().fp8q_quant_floor_min_m(k, sm_count, groups_per_cta, rows_per_cta, min_ctas_per_sm))
+
+
+def quant_act(x: torch.Tensor, variant: int = AUTO, row_major: bool = True, out=None, stream=None):
+    """x bf16 [M, K] -> (q uint8 [M, K], s_row fp32 [M, K/128] or None, s_kmajor fp32 [K/128, ceil16(M)])."""
+    m, k = x.shape
+    _need(x, torch.bfloat16, (m, k), "x")
+    g, mp = k // GROUP, m_pad(m)
+    if out is None:
+        q = torch.empty((m, k), dtype=torch.uint8, device=x.device)
+        s_row = torch.empty((m, g), dtype=torch.float32, device=x.device) if row_major else None
+        s_k = torch.empty((g, mp), dtype=torch.float32, device=x.device)
+    else:
+        q, s_row, s_k = out
+    lib = _lib.load()
+    if variant == AUTO:
+        st = lib.fp8q_quant_act(_p(x), _p(q), _p(s_row), _p(s_k), m, k, _stream(stream))
+    else:
+        st = lib.fp8q_quant_act_variant(_p(x), _p(q), _p(s_row), _p(s_k), m, k, variant, _stream(stream))
+    _lib.check(st, "fp8q_quant_act")
+    return q, s_row, s_k
+
+
+def quant_weight(w: torch.Tensor, stream=None):
+    """w bf16 [N, K] -> (wq uint8 [N, K], w_scale fp32 [N/128, K/128])."""
+    n, k = w.shape
+    _need(w, torch.bfloat16, (n, k), "w")
+    wq = torch.empty((n, k), dtype=torch.uint8, device=w.device)
+    ws = torch.empty((n // GROUP, k // GROUP), dtype=torch.float32, device=w.device)
+    _lib.check(_lib.load().fp8q_quant_weight(_p(w), _p(wq), _p(ws), n, k, _stream(stream)), "fp8q_quant_weight")
+    return wq, ws
+
+
+def gemm_blockscaled(q: torch.Tensor, s_kmajor: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
+                     out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """q uint8 [M,K], s_kmajor fp32 [K/128, ceil16(M)], wq uint8 [N,K], w_scale fp32 [N/128,K/128] -> y bf16 [M,N]."""
+    m, k = q.shape
+    n = wq.shape[0]
+    _need(q, torch.uint8, (m, k), "q")
+    _need(s_kmajor, torch.float32, (k // GROUP, m_pad(m)), "s_kmajor")
+    _need(wq, torch.uint8, (n, k), "wq")
+    _need(w_scale, torch.float32, (n // GROUP, k // GROUP), "w_scale")
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=q.device) if out is None else out
+    _need(y, torch.bfloat16, (m, n), "y")
+    _lib.check(_lib.load().fp8q_gemm_blockscaled(_p(q), _p(s_kmajor), _p(wq), _p(w_scale), _p(y), m, n, k,
+                                                  _stream(stream)), "fp8q_gemm_blockscaled")
+    return y
+
+
+def linear_workspace_bytes(m: int, k: int) -> int:
+    return int(_lib.load().fp8q_linear_workspace_bytes(m, k))
+
+
+def linear_scale_offset(m: int, k: int) -> int:
+    return int(_lib.load().fp8q_linear_scale_offset(m, k))
+
+
+def linear(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor, workspace: torch.Tensor | None = None,
+           out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Fused W8A8 linear: x bf16 [M,K] -> y bf16 [M,N] (quantize + block-scaled GEMM in one call)."""
+    m, k = x.shape
+    n = wq.shape[0]
+    _need(x, torch.bfloat16, (m, k), "x")
+    _need(wq, torch.uint8, (n, k), "wq")
+    _need(w_scale, torch.float32, (n // GROUP, k // GROUP), "w_scale")
+    need = linear_workspace_bytes(m, k)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _need(y, torch.bfloat16, (m, n), "y")
+    _lib.check(_lib.load().fp8q_linear(_p(x), _p(wq), _p(w_scale), _p(y), _p(workspace), workspace.numel(),
+                                        m, n, k, _stream(stream)), "fp8q_linear")
+    return y
+
+
+def convert_e4m3(t: torch.Tensor, stream=None) -> torch.Tensor:
+    """fp32 CUDA tensor -> uint8 e4m3 codes with the quantizers' conversion."""
+    if not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+        raise ValueError("t must be a contiguous fp32 CUDA tensor")
+    out = torch.empty(t.shape, dtype=torch.uint8, device=t.device)
+    _lib.check(_lib.load().fp8q_convert_e4m3(_p(t), _p(out), t.numel(), _stream(stream)), "fp8q_convert_e4m3")
+    return out
+
+
+def launch_count() -> int:
+    return int(_lib.load().fp8q_launch_count())
+
+
+def device_error(stream=None) -> int:
+    code = ctypes.c_uint32(0)
+    st = _lib.load().fp8q_device_error(_stream(stream), ctypes.byref(code))
+    if st not in (0, 6):
+        _lib.check(st, "fp8q_device_error")
+    return int(code.value)

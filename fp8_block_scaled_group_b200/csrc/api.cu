@@ -1,0 +1,283 @@
+// C ABI of libfp8q.so: argument checks, the quantizer variant pick, and the
+// launch sequence of each call. Declarations and contracts: include/fp8q.h.
+#include <atomic>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "fp8q.h"
+#include "internal.h"
+
+namespace fp8q {
+
+static std::atomic<uint64_t> g_launches{0};
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+namespace {
+
+constexpr uint32_t kGroup = 128;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+uint32_t ceil_div(uint32_t a, uint32_t b) { return (a + b - 1) / b; }
+
+// Per-device facts, queried once per device.
+struct DeviceInfo {
+    int major = -1, minor = -1, sms = 0;
+};
+
+fp8q_status current_device(DeviceInfo* out) {
+    static std::mutex mu;
+    static DeviceInfo cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return FP8Q_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    DeviceInfo& d = cache[dev];
+    if (d.major < 0) {
+        if (cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            d = DeviceInfo{};
+            cudaGetLastError();
+            return FP8Q_ERR_CUDA;
+        }
+    }
+    *out = d;
+    if (d.major != 10 || d.minor != 0) return FP8Q_ERR_UNSUPPORTED_DEVICE;
+    return FP8Q_OK;
+}
+
+// FP8Q_QUANT_VARIANT=single|multi forces a variant (read once).
+int32_t env_variant() {
+    static int32_t v = [] {
+        const char* e = std::getenv("FP8Q_QUANT_VARIANT");
+        if (!e) return static_cast<int32_t>(FP8Q_QUANT_AUTO);
+        if (!std::strcmp(e, "single")) return static_cast<int32_t>(FP8Q_QUANT_SINGLE);
+        if (!std::strcmp(e, "multi")) return static_cast<int32_t>(FP8Q_QUANT_MULTI);
+        return static_cast<int32_t>(FP8Q_QUANT_AUTO);
+    }();
+    return v;
+}
+
+// FP8Q_LOG=1: one line per process per pick branch, so a run that sees both
+// decode and prefill widths reports both variants once.
+void log_pick(const fp8q_quant_pick_t& p, uint32_t m, uint32_t k) {
+    static const bool on = [] {
+        const char* e = std::getenv("FP8Q_LOG");
+        return e && e[0] == '1';
+    }();
+    if (!on) return;
+    static std::atomic<bool> said[4];
+    const int slot = (p.variant == FP8Q_QUANT_MULTI ? 1 : 0) + (p.forced ? 2 : 0);
+    if (said[slot].exchange(true)) return;
+    std::fprintf(stderr,
+                 "fp8q: act-quant variant %s at M=%u K=%u grid=%u block=%u (multi grid %u CTAs, floor %u)%s\n",
+                 p.variant == FP8Q_QUANT_MULTI ? "multi" : "single", m, k, p.grid_x, p.block_x, p.multi_ctas,
+                 p.floor_ctas, p.forced ? " [forced]" : "");
+}
+
+// Shapes first; with M == 0 there is nothing to read or write, so the
+// pointers of empty buffers (possibly NULL) are accepted.
+fp8q_status check_quant_args(const void* x, const void* q, const float* s_row, const float* s_k, uint32_t m,
+                             uint32_t k) {
+    if (k == 0 || k % kGroup) return FP8Q_ERR_SHAPE;
+    if (m == 0) return FP8Q_OK;
+    if (!x || !q || !s_k) return FP8Q_ERR_NULL;
+    if (static_cast<uint64_t>(m) * k >= (1ull << 31)) return FP8Q_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(s_k) || (s_row && !aligned16(s_row))) return FP8Q_ERR_ALIGN;
+    return FP8Q_OK;
+}
+
+fp8q_status check_gemm_args(const void* q, const float* s_k, const void* wq, const float* w_s, const void* y,
+                            uint32_t m, uint32_t n, uint32_t k) {
+    if (k == 0 || k % kGroup || n == 0 || n % kGroup) return FP8Q_ERR_SHAPE;
+    if (m == 0) return FP8Q_OK;
+    if (!q || !s_k || !wq || !w_s || !y) return FP8Q_ERR_NULL;
+    if (static_cast<uint64_t>(m) * k >= (1ull << 31) || static_cast<uint64_t>(n) * k >= (1ull << 31) ||
+        static_cast<uint64_t>(m) * n >= (1ull << 31))
+        return FP8Q_ERR_SHAPE;
+    if (!aligned16(q) || !aligned16(s_k) || !aligned16(wq) || !aligned16(w_s) || !aligned16(y))
+        return FP8Q_ERR_ALIGN;
+    return FP8Q_OK;
+}
+
+fp8q_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return FP8Q_OK;
+    cudaGetLastError();
+    return FP8Q_ERR_CUDA;
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace
+}  // namespace fp8q
+
+using namespace fp8q;
+
+extern "C" {
+
+const char* fp8q_status_string(int status) {
+    switch (status) {
+        case FP8Q_OK: return "FP8Q_OK";
+        case FP8Q_ERR_NULL: return "FP8Q_ERR_NULL: a required pointer is NULL";
+        case FP8Q_ERR_SHAPE: return "FP8Q_ERR_SHAPE: K and N must be non-zero multiples of 128 and sizes below 2^31";
+        case FP8Q_ERR_ALIGN: return "FP8Q_ERR_ALIGN: pointers must be 16-byte aligned";
+        case FP8Q_ERR_WORKSPACE: return "FP8Q_ERR_WORKSPACE: workspace too small or misaligned";
+        case FP8Q_ERR_CUDA: return "FP8Q_ERR_CUDA: a CUDA call failed";
+        case FP8Q_ERR_DEVICE_TIMEOUT: return "FP8Q_ERR_DEVICE_TIMEOUT: a kernel gave up on a bounded wait";
+        case FP8Q_ERR_UNSUPPORTED_DEVICE: return "FP8Q_ERR_UNSUPPORTED_DEVICE: needs compute capability 10.0 (B200)";
+        case FP8Q_ERR_ARG: return "FP8Q_ERR_ARG: invalid argument";
+        default: return "FP8Q_ERR_UNKNOWN";
+    }
+}
+
+const char* fp8q_version(void) { return "fp8q 0.1.0 (sm_100a)"; }
+
+uint32_t fp8q_m_pad(uint32_t m) { return (m + 15u) / 16u * 16u; }
+
+uint32_t fp8q_quant_floor_min_m(uint32_t k, uint32_t sm_count, uint32_t groups_per_cta, uint32_t rows_per_cta,
+                                uint32_t min_ctas_per_sm) {
+    if (k < kGroup || groups_per_cta == 0 || rows_per_cta == 0) return 0;
+    const uint64_t grid_x = ceil_div(k / kGroup, groups_per_cta);
+    const uint64_t floor_ctas = static_cast<uint64_t>(min_ctas_per_sm) * (sm_count ? sm_count : 1u);
+    // smallest M with grid_x * ceil(M / rows_per_cta) >= floor_ctas
+    const uint64_t row_blocks = (floor_ctas + grid_x - 1) / grid_x;
+    const uint64_t min_m = row_blocks == 0 ? 0 : (row_blocks - 1) * rows_per_cta + 1;
+    return static_cast<uint32_t>(min_m > 0xFFFFFFFFull ? 0xFFFFFFFFull : min_m);
+}
+
+fp8q_status fp8q_quant_pick(uint32_t m, uint32_t k, uint32_t sm_count, int32_t requested,
+                            fp8q_quant_pick_t* out) {
+    if (!out) return FP8Q_ERR_NULL;
+    if (k == 0 || k % kGroup) return FP8Q_ERR_SHAPE;
+    if (sm_count == 0 || requested < FP8Q_QUANT_AUTO || requested > FP8Q_QUANT_MULTI) return FP8Q_ERR_ARG;
+    const uint32_t G = k / kGroup;
+    fp8q_quant_pick_t p;
+    std::memset(&p, 0, sizeof p);
+    const uint64_t multi = static_cast<uint64_t>(ceil_div(G, kMultiGroupsPerCta)) * ceil_div(m, kMultiRowsPerCta);
+    p.multi_ctas = static_cast<uint32_t>(multi > 0xFFFFFFFFull ? 0xFFFFFFFFull : multi);
+    p.floor_ctas = kMultiMinCtasPerSm * sm_count;
+    int32_t v;
+    if (requested == FP8Q_QUANT_AUTO) {
+        // The floor, read from the same function the tests and logs use, so
+        // it cannot disagree with the grid it guards.
+        const uint32_t min_m =
+            fp8q_quant_floor_min_m(k, sm_count, kMultiGroupsPerCta, kMultiRowsPerCta, kMultiMinCtasPerSm);
+        v = m >= min_m ? FP8Q_QUANT_MULTI : FP8Q_QUANT_SINGLE;
+    } else {
+        v = requested;
+        p.forced = 1;
+    }
+    p.variant = v;
+    if (v == FP8Q_QUANT_MULTI) {
+        p.grid_x = p.multi_ctas;
+        p.block_x = 128;
+        p.groups_per_cta = kMultiGroupsPerCta * kMultiRowsPerCta;
+    } else {
+        const uint64_t single = static_cast<uint64_t>(G) * m;
+        p.grid_x = static_cast<uint32_t>(single > 0xFFFFFFFFull ? 0xFFFFFFFFull : single);
+        p.block_x = 16;
+        p.groups_per_cta = 1;
+    }
+    *out = p;
+    return FP8Q_OK;
+}
+
+fp8q_status fp8q_quant_act_variant(const void* x, void* q, float* s_row, float* s_kmajor, uint32_t m, uint32_t k,
+                                   int32_t variant, void* stream) {
+    fp8q_status st = check_quant_args(x, q, s_row, s_kmajor, m, k);
+    if (st != FP8Q_OK) return st;
+    if (variant < FP8Q_QUANT_AUTO || variant > FP8Q_QUANT_MULTI) return FP8Q_ERR_ARG;
+    if (m == 0) return FP8Q_OK;
+    DeviceInfo dev;
+    if ((st = current_device(&dev)) != FP8Q_OK) return st;
+    fp8q_quant_pick_t pick;
+    if ((st = fp8q_quant_pick(m, k, static_cast<uint32_t>(dev.sms), variant, &pick)) != FP8Q_OK) return st;
+    log_pick(pick, m, k);
+    QuantLaunch L{x, q, s_row, s_kmajor, m, k, fp8q_m_pad(m), pick.variant};
+    return from_cuda(launch_quant_act(L, static_cast<cudaStream_t>(stream)));
+}
+
+fp8q_status fp8q_quant_act(const void* x, void* q, float* s_row, float* s_kmajor, uint32_t m, uint32_t k,
+                           void* stream) {
+    return fp8q_quant_act_variant(x, q, s_row, s_kmajor, m, k, env_variant(), stream);
+}
+
+fp8q_status fp8q_quant_weight(const void* w, void* wq, float* w_scale, uint32_t n, uint32_t k, void* stream) {
+    if (k == 0 || k % kGroup || n == 0 || n % kGroup) return FP8Q_ERR_SHAPE;
+    if (!w || !wq || !w_scale) return FP8Q_ERR_NULL;
+    if (static_cast<uint64_t>(n) * k >= (1ull << 31)) return FP8Q_ERR_SHAPE;
+    if (!aligned16(w) || !aligned16(wq) || !aligned16(w_scale)) return FP8Q_ERR_ALIGN;
+    DeviceInfo dev;
+    fp8q_status st = current_device(&dev);
+    if (st != FP8Q_OK) return st;
+    return from_cuda(launch_quant_weight(w, wq, w_scale, n, k, static_cast<cudaStream_t>(stream)));
+}
+
+fp8q_status fp8q_gemm_blockscaled(const void* q, const float* s_kmajor, const void* wq, const float* w_scale,
+                                  void* y, uint32_t m, uint32_t n, uint32_t k, void* stream) {
+    fp8q_status st = check_gemm_args(q, s_kmajor, wq, w_scale, y, m, n, k);
+    if (st != FP8Q_OK) return st;
+    if (m == 0) return FP8Q_OK;
+    DeviceInfo dev;
+    if ((st = current_device(&dev)) != FP8Q_OK) return st;
+    GemmLaunch L{q, s_kmajor, wq, w_scale, y, m, n, k, fp8q_m_pad(m)};
+    return from_cuda(launch_gemm(L, static_cast<cudaStream_t>(stream)));
+}
+
+size_t fp8q_linear_scale_offset(uint32_t m, uint32_t k) {
+    return round_up(static_cast<size_t>(m) * k, 256);
+}
+
+size_t fp8q_linear_workspace_bytes(uint32_t m, uint32_t k) {
+    const size_t g = k / kGroup;
+    return fp8q_linear_scale_offset(m, k) + round_up(g * fp8q_m_pad(m) * sizeof(float), 256);
+}
+
+fp8q_status fp8q_linear(const void* x, const void* wq, const float* w_scale, void* y, void* workspace,
+                        size_t workspace_bytes, uint32_t m, uint32_t n, uint32_t k, void* stream) {
+    if (k == 0 || k % kGroup || n == 0 || n % kGroup) return FP8Q_ERR_SHAPE;
+    if (m == 0) return FP8Q_OK;
+    if (!x || !wq || !w_scale || !y || !workspace) return FP8Q_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FP8Q_ERR_WORKSPACE;
+    if (workspace_bytes < fp8q_linear_workspace_bytes(m, k)) return FP8Q_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* s_k = reinterpret_cast<float*>(ws + fp8q_linear_scale_offset(m, k));
+    fp8q_status st = check_quant_args(x, ws, nullptr, s_k, m, k);
+    if (st != FP8Q_OK) return st;
+    if ((st = check_gemm_args(ws, s_k, wq, w_scale, y, m, n, k)) != FP8Q_OK) return st;
+    if (m == 0) return FP8Q_OK;
+    if ((st = fp8q_quant_act(x, ws, nullptr, s_k, m, k, stream)) != FP8Q_OK) return st;
+    return fp8q_gemm_blockscaled(ws, s_k, wq, w_scale, y, m, n, k, stream);
+}
+
+fp8q_status fp8q_convert_e4m3(const float* in, uint8_t* out, size_t count, void* stream) {
+    if (!in || !out) return FP8Q_ERR_NULL;
+    if (count == 0) return FP8Q_OK;
+    DeviceInfo dev;
+    fp8q_status st = current_device(&dev);
+    if (st != FP8Q_OK) return st;
+    return from_cuda(launch_convert_e4m3(in, out, count, static_cast<cudaStream_t>(stream)));
+}
+
+uint64_t fp8q_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+fp8q_status fp8q_device_error(void* stream, uint32_t* code) {
+    if (!code) return FP8Q_ERR_NULL;
+    *code = 0;
+    DeviceInfo dev;
+    fp8q_status st = current_device(&dev);
+    if (st != FP8Q_OK) return st;
+    if (read_clear_device_error(code, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return FP8Q_ERR_CUDA;
+    }
+    return *code ? FP8Q_ERR_DEVICE_TIMEOUT : FP8Q_OK;
+}
+
+}  // extern "C"

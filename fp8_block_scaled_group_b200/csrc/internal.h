@@ -1,0 +1,50 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace fp8q {
+
+// Quantizer variants (values match FP8Q_QUANT_SINGLE / FP8Q_QUANT_MULTI).
+constexpr int kVariantSingle = 1;
+constexpr int kVariantMulti = 2;
+
+// MULTI geometry: 8 K-groups per CTA (one per half-warp), each half-warp
+// quantizing kMultiRowsPerCta consecutive tokens.
+constexpr uint32_t kMultiGroupsPerCta = 8;
+constexpr uint32_t kMultiRowsPerCta = 2;
+// MULTI runs when its grid reaches this many CTAs per SM.
+constexpr uint32_t kMultiMinCtasPerSm = 2;
+
+struct QuantLaunch {
+    const void* x;
+    void* q;
+    float* s_row;
+    float* s_k;
+    uint32_t m, k, mp;
+    int variant;
+};
+
+cudaError_t launch_quant_act(const QuantLaunch& L, cudaStream_t stream);
+cudaError_t launch_quant_weight(const void* w, void* wq, float* w_scale, uint32_t n, uint32_t k,
+                                cudaStream_t stream);
+cudaError_t launch_convert_e4m3(const float* in, uint8_t* out, size_t n, cudaStream_t stream);
+
+struct GemmLaunch {
+    const void* q;
+    const float* s_k;
+    const void* wq;
+    const float* w_scale;
+    void* y;
+    uint32_t m, n, k, mp;
+};
+
+cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream);
+
+cudaError_t read_clear_device_error(uint32_t* code, cudaStream_t stream);
+
+void note_launch();
+
+}  // namespace fp8q

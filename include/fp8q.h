@@ -1,0 +1,212 @@
+/*
+ * fp8q — W8A8 FP8 block-scaled linear projection for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libfp8q.so. The operations follow the pages
+ *   "spark_model/layers/ops/dispatch_proj.rs"      (P-DP below) and
+ *   "spark_model/layers/ops/fp8_act_quant_floor.rs" (P-FL below):
+ *   - per-token, per-128-K-group FP8 E4M3 activation quantization with FP32
+ *     scales (P-DP, `cublas_fp8_proj`: "FP8 + per-[token,128-of-K] scales"),
+ *     with the scales stored both row-major [M, K/128] and K-major
+ *     [K/128, ceil16(M)] with zeroed pad rows (P-DP, `fp8_act_scale_to_kmajor`
+ *     and the ⚠ SCALE LAYOUT note of `cublas_fp8_proj_prequant`);
+ *   - a GEMM out[M,N] = act[M,K] @ weight^T over FP8 weights carrying FP32
+ *     per-128x128-block scales, bf16 out (P-DP, `cublas_fp8_proj_prequant`,
+ *     `dequant_fp8_bf16_into` for the weight-scale indexing);
+ *   - the fused linear that runs both in one call (P-DP, `cublas_fp8_proj`);
+ *   - the choice between the one-group-per-CTA and the multi-group-per-CTA
+ *     quantizer by a CTA-count floor (P-FL, module header and
+ *     `fp8_act_quant_hopper_reject`), re-derived for the device's SM count.
+ *
+ * Conventions shared by every call:
+ *   - Data pointers are DEVICE pointers owned by the caller, 16-byte aligned.
+ *     The library allocates no device memory.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls
+ *     only enqueue work; nothing synchronizes.
+ *   - bf16 is IEEE bfloat16; e4m3 is OCP FP8 E4M3FN (bias 7, max 448, NaN
+ *     only at S.1111.111). Matrices are row-major.
+ *   - K and N must be multiples of 128. M == 0 is accepted and launches
+ *     nothing (pointers may then be NULL). M*K, N*K and M*N must stay
+ *     below 2^31.
+ *   - Every argument is checked before anything is enqueued; a failed check
+ *     returns its status and leaves all buffers untouched.
+ *   - A device other than compute capability 10.0 returns
+ *     FP8Q_ERR_UNSUPPORTED_DEVICE; there is no fallback path.
+ *   - NaN or Inf in the inputs is outside the contract (results undefined).
+ */
+#ifndef FP8Q_H
+#define FP8Q_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP8Q_OK = 0,
+    FP8Q_ERR_NULL = 1,               /* a required pointer is NULL                 */
+    FP8Q_ERR_SHAPE = 2,              /* K or N not a multiple of 128, or too large */
+    FP8Q_ERR_ALIGN = 3,              /* a pointer is not 16-byte aligned           */
+    FP8Q_ERR_WORKSPACE = 4,          /* workspace smaller than required            */
+    FP8Q_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed          */
+    FP8Q_ERR_DEVICE_TIMEOUT = 6,     /* a kernel's bounded wait ran out            */
+    FP8Q_ERR_UNSUPPORTED_DEVICE = 7, /* current device is not sm_100               */
+    FP8Q_ERR_ARG = 8                 /* any other invalid argument                 */
+} fp8q_status;
+
+/* Human-readable name of a status code; never NULL. */
+const char *fp8q_status_string(int status);
+
+/* Library version string. */
+const char *fp8q_version(void);
+
+/* ceil16(m): the token extent of the K-major scales (P-DP, `cublas_fp8_m_pad`). */
+uint32_t fp8q_m_pad(uint32_t m);
+
+/* ------------------------------------------------------ variant pick ---- */
+
+/* Quantizer variants. SINGLE quantizes one 128-wide group per CTA; MULTI
+   quantizes 8 consecutive groups of a few consecutive tokens per CTA
+   (fp8q_quant_pick_t.groups_per_cta). Both emit the same bytes (P-FL: the
+   two quantizers of the pages emit identical bytes, so the choice is one of
+   speed only). */
+enum { FP8Q_QUANT_AUTO = 0, FP8Q_QUANT_SINGLE = 1, FP8Q_QUANT_MULTI = 2 };
+
+typedef struct {
+    int32_t variant;          /* FP8Q_QUANT_SINGLE or FP8Q_QUANT_MULTI       */
+    uint32_t grid_x;          /* CTAs launched                               */
+    uint32_t block_x;         /* threads per CTA                             */
+    uint32_t groups_per_cta;  /* 128-wide K groups one CTA quantizes         */
+    uint32_t multi_ctas;      /* CTAs the MULTI variant would launch         */
+    uint32_t floor_ctas;      /* the CTA floor MULTI must reach              */
+    int32_t forced;           /* 1 when `requested` overrode the floor       */
+} fp8q_quant_pick_t;
+
+/*
+ * The smallest M at which a multi-group quantizer whose CTA covers
+ * `groups_per_cta` K-groups of `rows_per_cta` tokens reaches
+ * `min_ctas_per_sm * sm_count` CTAs at this K. Its grid is
+ * ceil((K/128)/groups_per_cta) x ceil(M/rows_per_cta) CTAs; with
+ * rows_per_cta = 1 this is the pages' formula ceil(floor / grid_y)
+ * (P-FL, `fp8_quant_hopper_min_m` and the per-K table of the module header:
+ * 132 SMs, 8 groups, 2 CTAs/SM gives 53/44/16 at K = 5120/6144/17408).
+ * fp8q_quant_pick applies exactly this function. Pure host function.
+ * Returns 0 when k < 128 or groups_per_cta or rows_per_cta is 0.
+ */
+uint32_t fp8q_quant_floor_min_m(uint32_t k, uint32_t sm_count, uint32_t groups_per_cta, uint32_t rows_per_cta,
+                                uint32_t min_ctas_per_sm);
+
+/*
+ * Which quantizer variant runs for (m, k) on a device with `sm_count` SMs,
+ * and on what grid (P-FL, `Fp8QuantPick`: the kernel and its grid travel
+ * together). `requested` is FP8Q_QUANT_AUTO (apply the floor) or a variant
+ * to force. Pure host function; no device is touched.
+ * Errors: FP8Q_ERR_NULL (out), FP8Q_ERR_SHAPE (k % 128), FP8Q_ERR_ARG
+ * (unknown variant or sm_count == 0).
+ */
+fp8q_status fp8q_quant_pick(uint32_t m, uint32_t k, uint32_t sm_count, int32_t requested,
+                            fp8q_quant_pick_t *out);
+
+/* ---------------------------------------------------------- kernels ---- */
+
+/*
+ * Per-token-group activation quantization (P-DP, `cublas_fp8_proj`, first
+ * step; P-FL for the variant). For each token t < m and group g < k/128:
+ *   amax = max_j |x[t][128g+j]|,  s = max(amax, 1e-10f) / 448.0f  (fp32),
+ *   q[t][128g+j] = e4m3_rne_satfinite(x[t][128g+j] / s)            (fp32 div)
+ *   x         bf16 [m, k]                                  (input)
+ *   q         e4m3 [m, k]                                  (output)
+ *   s_row     fp32 [m, k/128] row-major; may be NULL to skip this layout
+ *   s_kmajor  fp32 [k/128, ceil16(m)]: s_kmajor[g][t] = s for t < m and
+ *             +0.0f for m <= t < ceil16(m)                 (output, required)
+ * The variant follows fp8q_quant_pick(m, k, <device SMs>, FP8Q_QUANT_AUTO)
+ * unless the environment variable FP8Q_QUANT_VARIANT=single|multi forces it.
+ * Errors: NULL, ALIGN, SHAPE, UNSUPPORTED_DEVICE, CUDA.
+ */
+fp8q_status fp8q_quant_act(const void *x, void *q, float *s_row, float *s_kmajor,
+                           uint32_t m, uint32_t k, void *stream);
+
+/* fp8q_quant_act with the variant chosen by the caller (FP8Q_QUANT_AUTO,
+   FP8Q_QUANT_SINGLE or FP8Q_QUANT_MULTI); the bytes written are identical. */
+fp8q_status fp8q_quant_act_variant(const void *x, void *q, float *s_row, float *s_kmajor,
+                                   uint32_t m, uint32_t k, int32_t variant, void *stream);
+
+/*
+ * Weight pre-quantization per 128x128 block (the block-scaled `Fp8Weight`
+ * of P-DP; scale indexing of `dequant_fp8_bf16_into`): for each block
+ * (bn, bg) the same amax / scale / RNE-satfinite steps as above, taken over
+ * the block's 128x128 values.
+ *   w        bf16 [n, k]              (input)
+ *   wq       e4m3 [n, k]              (output)
+ *   w_scale  fp32 [n/128, k/128]      (output), scale of element (r, c) at
+ *            w_scale[(r/128)*(k/128) + c/128]
+ * Errors: NULL, ALIGN, SHAPE, UNSUPPORTED_DEVICE, CUDA.
+ */
+fp8q_status fp8q_quant_weight(const void *w, void *wq, float *w_scale,
+                              uint32_t n, uint32_t k, void *stream);
+
+/*
+ * Block-scaled FP8 GEMM (P-DP, `cublas_fp8_proj_prequant`):
+ *   y[t][c] = bf16_rn( sum_g s_kmajor[g][t] * w_scale[c/128][g]
+ *                      * sum_{j<128} q[t][128g+j] * wq[c][128g+j] )
+ * with the inner sums from FP8 tensor-core MMA in fp32 and the scaled
+ * promotion in fp32.
+ *   q         e4m3 [m, k]               (input; rows >= m are never read)
+ *   s_kmajor  fp32 [k/128, ceil16(m)]   (input, as written by fp8q_quant_act)
+ *   wq        e4m3 [n, k], w_scale fp32 [n/128, k/128]        (inputs)
+ *   y         bf16 [m, n]               (output; exactly m rows are written)
+ * Errors: NULL, ALIGN, SHAPE, UNSUPPORTED_DEVICE, CUDA.
+ */
+fp8q_status fp8q_gemm_blockscaled(const void *q, const float *s_kmajor, const void *wq,
+                                  const float *w_scale, void *y,
+                                  uint32_t m, uint32_t n, uint32_t k, void *stream);
+
+/*
+ * Workspace bytes fp8q_linear needs for (m, k): the FP8 activation
+ * [m, k] at offset 0, then the K-major scales [k/128, ceil16(m)] fp32 at
+ * offset fp8q_linear_scale_offset(m, k).
+ */
+size_t fp8q_linear_workspace_bytes(uint32_t m, uint32_t k);
+size_t fp8q_linear_scale_offset(uint32_t m, uint32_t k);
+
+/*
+ * Fused W8A8 linear (P-DP, `cublas_fp8_proj`): quantize x exactly as
+ * fp8q_quant_act does (same bytes, same K-major scales, left in the
+ * workspace), then run fp8q_gemm_blockscaled into y. One call; the kernels
+ * are chained on `stream`.
+ *   x bf16 [m, k]; wq e4m3 [n, k]; w_scale fp32 [n/128, k/128]; y bf16 [m, n]
+ *   workspace: device memory of at least fp8q_linear_workspace_bytes(m, k),
+ *              256-byte aligned, owned by the caller.
+ * Errors: NULL, ALIGN, SHAPE, WORKSPACE, UNSUPPORTED_DEVICE, CUDA.
+ */
+fp8q_status fp8q_linear(const void *x, const void *wq, const float *w_scale, void *y,
+                        void *workspace, size_t workspace_bytes,
+                        uint32_t m, uint32_t n, uint32_t k, void *stream);
+
+/* ------------------------------------------------------- diagnostics ---- */
+
+/*
+ * Convert `count` fp32 values to e4m3 codes with the same device routine
+ * the quantizers use (round-to-nearest-even, saturating at 448). Used to
+ * check the conversion exhaustively. Device pointers.
+ * Errors: NULL, UNSUPPORTED_DEVICE, CUDA.
+ */
+fp8q_status fp8q_convert_e4m3(const float *in, uint8_t *out, size_t count, void *stream);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t fp8q_launch_count(void);
+
+/*
+ * Read and clear the device error word of the current device: non-zero when
+ * a kernel's bounded wait ran out (the kernel then stopped early and its
+ * outputs are incomplete). Synchronizes `stream` first. Returns FP8Q_OK or
+ * FP8Q_ERR_DEVICE_TIMEOUT (with *code set), or FP8Q_ERR_CUDA.
+ */
+fp8q_status fp8q_device_error(void *stream, uint32_t *code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8Q_H */

@@ -1,0 +1,184 @@
+"""Host-side logic of libfp8q.so, exercised without a GPU.
+
+Covers: every symbol declared in include/fp8q.h is exported and bound; the
+CTA-floor function reproduces the worked table of the page
+"spark_model/layers/ops/fp8_act_quant_floor.rs" and the sign of its fifteen
+measured arms; the pick keeps kernel and grid together; argument checks
+return their status before anything touches a device.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from conftest import ROOT, golden_rows
+from fp8_block_scaled_group_b200 import _lib, api
+
+HEADER = os.path.join(ROOT, "include", "fp8q.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp8q_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ["fp8q_quant_act", "fp8q_gemm_blockscaled", "fp8q_linear", "fp8q_m_pad",
+                 "fp8q_quant_pick", "fp8q_quant_weight", "fp8q_status_string"]:
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    names = declared_functions()
+    for name in names:
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, f"{name} has no ctypes binding"
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (fp8q_\w+)", out))
+    assert set(names) <= exported
+    assert set(_lib.SIGNATURES) == set(names)
+
+
+def test_status_strings_and_version():
+    lib = _lib.load()
+    for code in range(0, 9):
+        s = lib.fp8q_status_string(code).decode()
+        assert s.startswith("FP8Q_")
+    assert lib.fp8q_status_string(99).decode() == "FP8Q_ERR_UNKNOWN"
+    assert b"sm_100a" in lib.fp8q_version()
+
+
+@pytest.mark.parametrize("m,mp", [(0, 0), (1, 16), (15, 16), (16, 16), (17, 32), (25, 32), (1168, 1168),
+                                  (4576, 4576), (4577, 4592)])
+def test_m_pad(m, mp):
+    assert api.m_pad(m) == mp
+
+
+def test_floor_reproduces_the_pages_table():
+    """sm_count 132, 8 K-groups per CTA, one token per CTA row, 2 CTAs per SM."""
+    for k, g, grid_y, min_m in (map(int, r) for r in golden_rows("cta_floor_h100.txt")):
+        assert k // 128 == g and -(-g // 8) == grid_y
+        assert api.quant_floor_min_m(k, 132, 8, 1, 2) == min_m
+
+
+def test_floor_reproduces_the_sign_of_fifteen_arms():
+    """The arm the floor picks is the arm measured faster, at every one of the 15 arms."""
+    rows = golden_rows("quant_arms_h100.txt")
+    assert len(rows) == 15
+    for m, k, faster in rows:
+        m, k = int(m), int(k)
+        picks_multi = m >= api.quant_floor_min_m(k, 132, 8, 1, 2)
+        assert picks_multi == (faster == "multi"), (m, k)
+
+
+def test_floor_rows_per_cta_generalisation():
+    # min M with ceil(G/8) * ceil(M/rpc) >= floor, checked by brute force
+    for k in [128, 512, 5120, 6144, 17408]:
+        for sms in [1, 132, 148]:
+            for rpc in [1, 2, 4]:
+                mm = api.quant_floor_min_m(k, sms, 8, rpc, 2)
+                gy = -(-(k // 128) // 8)
+                ok = [m for m in range(1, 5000) if gy * -(-m // rpc) >= 2 * sms]
+                assert mm == ok[0], (k, sms, rpc)
+    assert api.quant_floor_min_m(64, 148, 8, 1, 2) == 0
+    assert api.quant_floor_min_m(5120, 148, 0, 1, 2) == 0
+
+
+def test_pick_keeps_kernel_and_grid_together():
+    for m in [1, 16, 17, 25, 53, 60, 100, 1168, 4576]:
+        for k in [512, 5120, 6144, 17408]:
+            auto = api.quant_pick(m, k, 148)
+            g = k // 128
+            min_m = api.quant_floor_min_m(k, 148, 8, 2, 2)
+            assert auto.variant == (api.MULTI if m >= min_m else api.SINGLE)
+            assert auto.forced == 0
+            assert auto.floor_ctas == 2 * 148
+            assert auto.multi_ctas == -(-g // 8) * -(-m // 2)
+            single = api.quant_pick(m, k, 148, api.SINGLE)
+            assert single.variant == api.SINGLE and single.forced == 1
+            assert single.grid_x == m * g and single.block_x == 16 and single.groups_per_cta == 1
+            multi = api.quant_pick(m, k, 148, api.MULTI)
+            assert multi.variant == api.MULTI and multi.grid_x == multi.multi_ctas and multi.block_x == 128
+            assert multi.groups_per_cta == 16
+
+
+def test_pick_argument_errors():
+    lib = _lib.load()
+    out = _lib.QuantPick()
+    assert lib.fp8q_quant_pick(16, 5120, 148, 0, None) == 1
+    assert lib.fp8q_quant_pick(16, 5000, 148, 0, ctypes.byref(out)) == 2
+    assert lib.fp8q_quant_pick(16, 5120, 0, 0, ctypes.byref(out)) == 8
+    assert lib.fp8q_quant_pick(16, 5120, 148, 3, ctypes.byref(out)) == 8
+
+
+def test_workspace_layout():
+    for m, k in [(1, 128), (16, 512), (17, 5120), (25, 17408), (4576, 17408)]:
+        off = api.linear_scale_offset(m, k)
+        assert off >= m * k and off % 256 == 0
+        assert api.linear_workspace_bytes(m, k) >= off + 4 * (k // 128) * api.m_pad(m)
+        assert api.linear_workspace_bytes(m, k) % 256 == 0
+
+
+# Argument checks come first, so these run without any device.
+A = ctypes.c_void_p(0x10000)   # 16-byte aligned stand-ins, never dereferenced
+B = ctypes.c_void_p(0x20000)
+C = ctypes.c_void_p(0x30000)
+D = ctypes.c_void_p(0x40000)
+E = ctypes.c_void_p(0x50000)
+ODD = ctypes.c_void_p(0x10008)
+
+
+def test_quant_act_argument_errors():
+    lib = _lib.load()
+    assert lib.fp8q_quant_act(None, B, C, D, 16, 512, None) == 1
+    assert lib.fp8q_quant_act(A, None, C, D, 16, 512, None) == 1
+    assert lib.fp8q_quant_act(A, B, C, None, 16, 512, None) == 1
+    assert lib.fp8q_quant_act(A, B, C, D, 16, 500, None) == 2
+    assert lib.fp8q_quant_act(A, B, C, D, 16, 0, None) == 2
+    assert lib.fp8q_quant_act(A, B, C, D, 1 << 20, 1 << 12, None) == 2
+    assert lib.fp8q_quant_act(ODD, B, C, D, 16, 512, None) == 3
+    assert lib.fp8q_quant_act(A, B, ODD, D, 16, 512, None) == 3
+    assert lib.fp8q_quant_act_variant(A, B, C, D, 16, 512, 7, None) == 8
+    assert lib.fp8q_quant_act(A, B, None, D, 0, 512, None) == 0  # M == 0: nothing to do
+    assert lib.fp8q_quant_act(None, None, None, None, 0, 512, None) == 0
+    assert lib.fp8q_quant_act(None, None, None, None, 0, 500, None) == 2
+
+
+def test_gemm_and_linear_argument_errors():
+    lib = _lib.load()
+    assert lib.fp8q_gemm_blockscaled(None, B, C, D, E, 16, 256, 512, None) == 1
+    assert lib.fp8q_gemm_blockscaled(A, B, C, D, None, 16, 256, 512, None) == 1
+    assert lib.fp8q_gemm_blockscaled(None, None, None, None, None, 0, 256, 512, None) == 0
+    assert lib.fp8q_gemm_blockscaled(A, B, C, D, E, 16, 200, 512, None) == 2
+    assert lib.fp8q_gemm_blockscaled(A, B, C, D, E, 16, 256, 520, None) == 2
+    assert lib.fp8q_gemm_blockscaled(A, B, C, D, ODD, 16, 256, 512, None) == 3
+    assert lib.fp8q_gemm_blockscaled(A, B, C, D, E, 0, 256, 512, None) == 0
+    need = lib.fp8q_linear_workspace_bytes(16, 512)
+    ws = ctypes.c_void_p(0x100000)
+    assert lib.fp8q_linear(A, B, C, D, None, need, 16, 256, 512, None) == 1
+    assert lib.fp8q_linear(None, None, None, None, None, 0, 0, 256, 512, None) == 0
+    assert lib.fp8q_linear(A, B, C, D, ws, need - 1, 16, 256, 512, None) == 4
+    assert lib.fp8q_linear(A, B, C, D, ctypes.c_void_p(0x100010), need, 16, 256, 512, None) == 4
+    assert lib.fp8q_linear(A, B, C, D, ws, need, 16, 256, 500, None) == 2
+    assert lib.fp8q_linear(A, B, C, D, ws, need, 0, 256, 512, None) == 0
+    assert lib.fp8q_quant_weight(A, B, None, 256, 512, None) == 1
+    assert lib.fp8q_quant_weight(A, B, C, 200, 512, None) == 2
+    assert lib.fp8q_quant_weight(ODD, B, C, 256, 512, None) == 3
+    assert lib.fp8q_convert_e4m3(None, B, 4, None) == 1
+    assert lib.fp8q_convert_e4m3(A, B, 0, None) == 0
+
+
+def test_no_device_reports_cuda_error_not_crash():
+    """With valid arguments and no usable device, calls fail with a status."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    lib = _lib.load()
+    assert lib.fp8q_quant_act(A, B, C, D, 16, 512, None) in (5, 7)
+    code = ctypes.c_uint32(0)
+    assert lib.fp8q_device_error(None, ctypes.byref(code)) in (5, 7)
