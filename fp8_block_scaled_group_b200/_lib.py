@@ -49,6 +49,7 @@ SIGNATURES = {
     "fp8q_linear_workspace_bytes": (SZ, [U32, U32]),
     "fp8q_linear_scale_offset": (SZ, [U32, U32]),
     "fp8q_linear": (ctypes.c_int, [P, P, P, P, P, SZ, U32, U32, U32, P]),
+    "fp8q_linear_noalloc": (ctypes.c_int, [P, P, P, P, U32, U32, U32, P]),
     "fp8q_convert_e4m3": (ctypes.c_int, [P, P, SZ, P]),
     "fp8q_launch_count": (ctypes.c_uint64, []),
     "fp8q_device_error": (ctypes.c_int, [P, ctypes.POINTER(ctypes.c_uint32)]),

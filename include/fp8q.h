@@ -184,6 +184,34 @@ fp8q_status fp8q_linear(const void *x, const void *wq, const float *w_scale, voi
                         void *workspace, size_t workspace_bytes,
                         uint32_t m, uint32_t n, uint32_t k, void *stream);
 
+/*
+ * fp8q_linear for callers that cannot allocate device memory. The paper has
+ * no counterpart to this call; it exists for callers that are handed inputs
+ * and outputs but cannot obtain a device buffer for the workspace: a plugin
+ * inside a runtime that owns the whole device-memory budget, or a
+ * latency-critical loop where a cudaMalloc could synchronize the device.
+ *
+ * Same arguments, results and kernels as fp8q_linear, minus the workspace:
+ * the FP8 activation and its K-major scales go to a fixed 16 MiB device
+ * array inside the library (every GPU that loads the library holds it until
+ * the process exits). The call allocates nothing and calls no allocating
+ * routine.
+ *   - Limit: fp8q_linear_workspace_bytes(m, k) must be at most 16 MiB
+ *     (about m*k <= 16.2 million, e.g. m = 1168 at k = 5120); larger calls
+ *     return FP8Q_ERR_WORKSPACE without enqueuing anything.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one array and it keeps the last
+ *     call's contents; nothing in it needs clearing, because each call
+ *     overwrites all of it that it reads. Calls that overlap on the GPU
+ *     (different streams, or different host threads, on one device) race on
+ *     the array: serialize them.
+ * Errors: NULL, ALIGN, SHAPE, WORKSPACE (too large), UNSUPPORTED_DEVICE, CUDA.
+ */
+fp8q_status fp8q_linear_noalloc(const void *x, const void *wq, const float *w_scale, void *y,
+                                uint32_t m, uint32_t n, uint32_t k, void *stream);
+
 /* ------------------------------------------------------- diagnostics ---- */
 
 /*
