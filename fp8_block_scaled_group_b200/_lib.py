@@ -40,7 +40,7 @@ SIGNATURES = {
     "fp8q_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fp8q_version": (ctypes.c_char_p, []),
     "fp8q_m_pad": (U32, [U32]),
-    "fp8q_quant_floor_min_m": (U32, [U32, U32, U32, U32, U32]),
+    "fp8q_quant_floor_min_m": (U32, [U32, U32, U32, U32, ctypes.c_float]),
     "fp8q_quant_pick": (ctypes.c_int, [U32, U32, U32, I32, ctypes.POINTER(QuantPick)]),
     "fp8q_quant_act": (ctypes.c_int, [P, P, P, P, U32, U32, P]),
     "fp8q_quant_act_variant": (ctypes.c_int, [P, P, P, P, U32, U32, I32, P]),
@@ -51,6 +51,7 @@ SIGNATURES = {
     "fp8q_linear": (ctypes.c_int, [P, P, P, P, P, SZ, U32, U32, U32, P]),
     "fp8q_linear_noalloc": (ctypes.c_int, [P, P, P, P, U32, U32, U32, P]),
     "fp8q_convert_e4m3": (ctypes.c_int, [P, P, SZ, P]),
+    "fp8q_check_division": (ctypes.c_int, [P, P]),
     "fp8q_launch_count": (ctypes.c_uint64, []),
     "fp8q_device_error": (ctypes.c_int, [P, ctypes.POINTER(ctypes.c_uint32)]),
 }

@@ -47,7 +47,8 @@ def quant_pick(m: int, k: int, sm_count: int, requested: int = AUTO) -> _lib.Qua
     return out
 
 
-def quant_floor_min_m(k: int, sm_count: int, groups_per_cta: int, rows_per_cta: int, min_ctas_per_sm: int) -> int:
+def quant_floor_min_m(k: int, sm_count: int, groups_per_cta: int, rows_per_cta: int,
+                      min_ctas_per_sm: float) -> int:
     return int(_lib.load().fp8q_quant_floor_min_m(k, sm_count, groups_per_cta, rows_per_cta, min_ctas_per_sm))
 
 
@@ -130,6 +131,14 @@ def convert_e4m3(t: torch.Tensor, stream=None) -> torch.Tensor:
     out = torch.empty(t.shape, dtype=torch.uint8, device=t.device)
     _lib.check(_lib.load().fp8q_convert_e4m3(_p(t), _p(out), t.numel(), _stream(stream)), "fp8q_convert_e4m3")
     return out
+
+
+def check_division(stream=None) -> tuple[int, int, int]:
+    """Run the exhaustive division check; returns (pairs, code mismatches, quotient mismatches)."""
+    counts = torch.zeros(3, dtype=torch.int64, device="cuda")
+    _lib.check(_lib.load().fp8q_check_division(_p(counts), _stream(stream)), "fp8q_check_division")
+    a, b, c = counts.cpu().tolist()
+    return int(a), int(b), int(c)
 
 
 def launch_count() -> int:

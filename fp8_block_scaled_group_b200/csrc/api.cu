@@ -1,6 +1,7 @@
 // C ABI of libfp8q.so: argument checks, the quantizer variant pick, and the
 // launch sequence of each call. Declarations and contracts: include/fp8q.h.
 #include <atomic>
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -114,6 +115,12 @@ fp8q_status from_cuda(cudaError_t e) {
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// ceil(min_ctas_per_sm * sm_count), at least 1.
+uint64_t floor_cta_count(uint32_t sm_count, float min_ctas_per_sm) {
+    const double f = std::ceil(static_cast<double>(min_ctas_per_sm) * (sm_count ? sm_count : 1u) - 1e-9);
+    return f < 1.0 ? 1u : static_cast<uint64_t>(f);
+}
+
 }  // namespace
 }  // namespace fp8q
 
@@ -141,10 +148,10 @@ const char* fp8q_version(void) { return "fp8q 0.1.0 (sm_100a)"; }
 uint32_t fp8q_m_pad(uint32_t m) { return (m + 15u) / 16u * 16u; }
 
 uint32_t fp8q_quant_floor_min_m(uint32_t k, uint32_t sm_count, uint32_t groups_per_cta, uint32_t rows_per_cta,
-                                uint32_t min_ctas_per_sm) {
-    if (k < kGroup || groups_per_cta == 0 || rows_per_cta == 0) return 0;
+                                float min_ctas_per_sm) {
+    if (k < kGroup || groups_per_cta == 0 || rows_per_cta == 0 || !(min_ctas_per_sm >= 0.0f)) return 0;
     const uint64_t grid_x = ceil_div(k / kGroup, groups_per_cta);
-    const uint64_t floor_ctas = static_cast<uint64_t>(min_ctas_per_sm) * (sm_count ? sm_count : 1u);
+    const uint64_t floor_ctas = floor_cta_count(sm_count, min_ctas_per_sm);
     // smallest M with grid_x * ceil(M / rows_per_cta) >= floor_ctas
     const uint64_t row_blocks = (floor_ctas + grid_x - 1) / grid_x;
     const uint64_t min_m = row_blocks == 0 ? 0 : (row_blocks - 1) * rows_per_cta + 1;
@@ -161,7 +168,7 @@ fp8q_status fp8q_quant_pick(uint32_t m, uint32_t k, uint32_t sm_count, int32_t r
     std::memset(&p, 0, sizeof p);
     const uint64_t multi = static_cast<uint64_t>(ceil_div(G, kMultiGroupsPerCta)) * ceil_div(m, kMultiRowsPerCta);
     p.multi_ctas = static_cast<uint32_t>(multi > 0xFFFFFFFFull ? 0xFFFFFFFFull : multi);
-    p.floor_ctas = kMultiMinCtasPerSm * sm_count;
+    p.floor_ctas = static_cast<uint32_t>(floor_cta_count(sm_count, kMultiMinCtasPerSm));
     int32_t v;
     if (requested == FP8Q_QUANT_AUTO) {
         // The floor, read from the same function the tests and logs use, so
@@ -176,7 +183,7 @@ fp8q_status fp8q_quant_pick(uint32_t m, uint32_t k, uint32_t sm_count, int32_t r
     p.variant = v;
     if (v == FP8Q_QUANT_MULTI) {
         p.grid_x = p.multi_ctas;
-        p.block_x = 128;
+        p.block_x = 64;
         p.groups_per_cta = kMultiGroupsPerCta * kMultiRowsPerCta;
     } else {
         const uint64_t single = static_cast<uint64_t>(G) * m;
@@ -263,6 +270,14 @@ fp8q_status fp8q_convert_e4m3(const float* in, uint8_t* out, size_t count, void*
     fp8q_status st = current_device(&dev);
     if (st != FP8Q_OK) return st;
     return from_cuda(launch_convert_e4m3(in, out, count, static_cast<cudaStream_t>(stream)));
+}
+
+fp8q_status fp8q_check_division(unsigned long long* counts, void* stream) {
+    if (!counts) return FP8Q_ERR_NULL;
+    DeviceInfo dev;
+    fp8q_status st = current_device(&dev);
+    if (st != FP8Q_OK) return st;
+    return from_cuda(launch_check_division(counts, static_cast<cudaStream_t>(stream)));
 }
 
 uint64_t fp8q_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

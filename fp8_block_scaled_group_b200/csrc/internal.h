@@ -11,12 +11,14 @@ namespace fp8q {
 constexpr int kVariantSingle = 1;
 constexpr int kVariantMulti = 2;
 
-// MULTI geometry: 8 K-groups per CTA (one per half-warp), each half-warp
-// quantizing kMultiRowsPerCta consecutive tokens.
+// MULTI geometry: 8 K-groups per CTA (eight lanes each), each quantized
+// for kMultiRowsPerCta consecutive tokens.
 constexpr uint32_t kMultiGroupsPerCta = 8;
-constexpr uint32_t kMultiRowsPerCta = 2;
-// MULTI runs when its grid reaches this many CTAs per SM.
-constexpr uint32_t kMultiMinCtasPerSm = 2;
+constexpr uint32_t kMultiRowsPerCta = 4;
+// MULTI runs when its grid reaches this many CTAs per SM (B200 sweep of
+// both variants over M in 1..4576 at K = 5120, 6144, 17408: MULTI overtakes
+// SINGLE once its grid holds about two thirds of a CTA per SM).
+constexpr float kMultiMinCtasPerSm = 2.0f / 3.0f;
 
 struct QuantLaunch {
     const void* x;
@@ -31,6 +33,7 @@ cudaError_t launch_quant_act(const QuantLaunch& L, cudaStream_t stream);
 cudaError_t launch_quant_weight(const void* w, void* wq, float* w_scale, uint32_t n, uint32_t k,
                                 cudaStream_t stream);
 cudaError_t launch_convert_e4m3(const float* in, uint8_t* out, size_t n, cudaStream_t stream);
+cudaError_t launch_check_division(unsigned long long* counts, cudaStream_t stream);
 
 struct GemmLaunch {
     const void* q;

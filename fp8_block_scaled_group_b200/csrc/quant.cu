@@ -5,10 +5,11 @@
 // per token and per 128-wide K group, amax = max |x|, s = max(amax, 1e-10)/448
 // (IEEE fp32 division), q = e4m3 RNE-satfinite of x/s (IEEE fp32 division).
 //
-// Both activation variants are one HBM stream. A 128-element group is owned
-// by 16 lanes holding 8 bf16 each (one 16-byte load); amax is reduced with
-// four xor-shuffles inside the 16 lanes; each lane stores its 8 codes as one
-// 8-byte store, so a group's 128 codes leave as one contiguous 128-byte run.
+// Both activation variants are one HBM stream. In SINGLE a 128-element group
+// is owned by 16 lanes holding 8 bf16 each (one 16-byte load), in MULTI by 8
+// lanes holding 16; amax is reduced with xor-shuffles inside those lanes and
+// each lane stores its codes as 8-byte stores, so a group's 128 codes leave
+// as contiguous runs.
 // The scale goes to the row-major [M, K/128] buffer and, in the same kernel,
 // to the K-major [K/128, ceil16(M)] buffer, whose pad rows the same launch
 // zero-fills; the pages spend a separate transpose launch on that layout
@@ -16,8 +17,9 @@
 //
 //   SINGLE: one group per CTA (16 threads), grid (K/128, M).
 //   MULTI : 8 consecutive groups of RPC consecutive tokens per CTA
-//           (128 threads), grid (ceil((K/128)/8), ceil(M/RPC)). Each lane
-//           keeps RPC independent 16-byte loads in flight.
+//           (64 threads, 8 lanes per group), grid (ceil((K/128)/8),
+//           ceil(M/RPC)). Each lane keeps 2*RPC independent 16-byte loads
+//           in flight.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -49,11 +51,14 @@ __device__ __forceinline__ void widen8(const uint4 v, float (&f)[8]) {
     f[7] = __uint_as_float(v.w & 0xFFFF0000u);
 }
 
-__device__ __forceinline__ float absmax8(const float (&f)[8]) {
-    float a = fabsf(f[0]);
-#pragma unroll
-    for (int i = 1; i < 8; ++i) a = fmaxf(a, fabsf(f[i]));
-    return a;
+// |x| maximum of 8 packed bf16, as fp32. With the sign bits cleared, finite
+// non-negative IEEE values order like their bit patterns, so the maximum is
+// taken on the integers, two 16-bit lanes at a time.
+__device__ __forceinline__ float absmax8_bits(const uint4 v) {
+    const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                                __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+    const uint32_t hi = m >> 16, lo = m & 0xFFFFu;
+    return __uint_as_float((hi > lo ? hi : lo) << 16);
 }
 
 // The scale of a group with absolute maximum `amax`: one fp32 division.
@@ -61,13 +66,31 @@ __device__ __forceinline__ float group_scale(float amax) {
     return __fdiv_rn(fmaxf(amax, 1e-10f), 448.0f);
 }
 
-// 8 values / s (IEEE division each) -> 8 codes packed little-endian.
+// x / s for a pair of values, rounded to nearest even, from the correctly
+// rounded reciprocal r = RN(1/s) and one remainder correction (Markstein's
+// division scheme, P. Markstein, IBM J. Res. Dev. 34(1), 1990):
+//   q0 = RN(x * r),  e = RN(x - q0 * s) (exact with a fused multiply-add),
+//   q  = RN(q0 + e * r).
+// The sign of x is put back at the end so that -0 stays -0. For every pair
+// (x, amax) of bf16 values with |x| <= amax, the code this gives equals the
+// code of the IEEE quotient: fp8q_check_division verifies it exhaustively on
+// the device.
+__device__ __forceinline__ float2 div2_by_scale(float2 x, float s, float r) {
+    const float2 q0 = __fmul2_rn(x, make_float2(r, r));
+    const float2 e = __ffma2_rn(make_float2(-q0.x, -q0.y), make_float2(s, s), x);
+    const float2 q = __ffma2_rn(e, make_float2(r, r), q0);
+    return make_float2(__uint_as_float(__float_as_uint(q.x) | (__float_as_uint(x.x) & 0x80000000u)),
+                       __uint_as_float(__float_as_uint(q.y) | (__float_as_uint(x.y) & 0x80000000u)));
+}
+
+// 8 values / s -> 8 codes packed little-endian.
 __device__ __forceinline__ uint2 encode8(const float (&f)[8], float s) {
+    const float r = __frcp_rn(s);
     uint32_t c[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint16_t p = cvt_e4m3x2(__fdiv_rn(f[2 * i], s), __fdiv_rn(f[2 * i + 1], s));
-        c[i] = p;
+        const float2 q = div2_by_scale(make_float2(f[2 * i], f[2 * i + 1]), s, r);
+        c[i] = cvt_e4m3x2(q.x, q.y);
     }
     return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
@@ -94,9 +117,10 @@ __global__ void __launch_bounds__(16) quant_act_single_kernel(const uint16_t* __
     const uint32_t g = blockIdx.x, t = blockIdx.y;
     const uint32_t lane = threadIdx.x;
     const size_t off = static_cast<size_t>(t) * k + static_cast<size_t>(g) * 128 + lane * 8;
+    const uint4 v = ld_stream16(x + off);
     float f[8];
-    widen8(ld_stream16(x + off), f);
-    float amax = absmax8(f);
+    widen8(v, f);
+    float amax = absmax8_bits(v);
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0x0000FFFFu, amax, o));
     const float s = group_scale(amax);
@@ -108,41 +132,55 @@ __global__ void __launch_bounds__(16) quant_act_single_kernel(const uint16_t* __
     zero_kmajor_pad(s_k, m, mp, G);
 }
 
-// MULTI: blockDim 128 (8 half-warps), grid (ceil(G/8), ceil(m/RPC)).
-// Half-warp h of CTA (bx, by) owns group g = 8*bx + h for tokens
-// RPC*by .. RPC*by + RPC - 1. Out-of-range groups/tokens compute on zeros
-// (so every shuffle sees its full warp) and store nothing.
+// MULTI: blockDim 64, grid (ceil(G/8), ceil(m/RPC)). Eight lanes own one
+// group: lane l holds elements 8l..8l+7 and 64+8l..64+8l+7 of it (two 16-byte
+// loads, each instruction covering the group's 128 contiguous bytes), so the
+// per-group work (scale, reciprocal, shuffles, scale stores) is shared by 16
+// elements per lane. Octet o of CTA (bx, by) owns group g = 8*bx + o for
+// tokens RPC*by .. RPC*by + RPC - 1; every load of the CTA is issued before
+// any arithmetic. Token validity is the same for the whole CTA, so rows past
+// m are skipped outright; a group past G (K/128 not a multiple of 8) computes
+// on zeros, so the shuffles still see their full warp, and stores nothing.
 template <int RPC>
-__global__ void __launch_bounds__(128) quant_act_multi_kernel(const uint16_t* __restrict__ x,
-                                                             uint8_t* __restrict__ q, float* __restrict__ s_row,
-                                                             float* __restrict__ s_k, uint32_t m, uint32_t k,
-                                                             uint32_t mp) {
+__global__ void __launch_bounds__(64) quant_act_multi_kernel(const uint16_t* __restrict__ x,
+                                                            uint8_t* __restrict__ q, float* __restrict__ s_row,
+                                                            float* __restrict__ s_k, uint32_t m, uint32_t k,
+                                                            uint32_t mp) {
     const uint32_t G = k >> 7;
-    const uint32_t lane = threadIdx.x & 15;
-    const uint32_t g = blockIdx.x * 8 + (threadIdx.x >> 4);
+    const uint32_t lane = threadIdx.x & 7;
+    const uint32_t g = blockIdx.x * 8 + (threadIdx.x >> 3);
     const uint32_t t0 = blockIdx.y * RPC;
     const bool g_ok = g < G;
-    uint4 v[RPC];
+    const uint32_t rows = m - t0 < static_cast<uint32_t>(RPC) ? m - t0 : static_cast<uint32_t>(RPC);
+    uint4 v[RPC][2];
 #pragma unroll
     for (int r = 0; r < RPC; ++r) {
-        const uint32_t t = t0 + r;
-        if (g_ok && t < m)
-            v[r] = ld_stream16(x + static_cast<size_t>(t) * k + static_cast<size_t>(g) * 128 + lane * 8);
-        else
-            v[r] = make_uint4(0u, 0u, 0u, 0u);
+        if (g_ok && static_cast<uint32_t>(r) < rows) {
+            const uint16_t* src = x + static_cast<size_t>(t0 + r) * k + static_cast<size_t>(g) * 128 + lane * 8;
+            v[r][0] = ld_stream16(src);
+            v[r][1] = ld_stream16(src + 64);
+        } else {
+            v[r][0] = make_uint4(0u, 0u, 0u, 0u);
+            v[r][1] = make_uint4(0u, 0u, 0u, 0u);
+        }
     }
 #pragma unroll
     for (int r = 0; r < RPC; ++r) {
+        if (static_cast<uint32_t>(r) >= rows) break;
         const uint32_t t = t0 + r;
-        float f[8];
-        widen8(v[r], f);
-        float amax = absmax8(f);
+        float amax = fmaxf(absmax8_bits(v[r][0]), absmax8_bits(v[r][1]));
 #pragma unroll
-        for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
         const float s = group_scale(amax);
-        const uint2 codes = encode8(f, s);
-        if (g_ok && t < m) {
-            st_stream8(q + static_cast<size_t>(t) * k + static_cast<size_t>(g) * 128 + lane * 8, codes);
+        float f0[8], f1[8];
+        widen8(v[r][0], f0);
+        widen8(v[r][1], f1);
+        const uint2 c0 = encode8(f0, s);
+        const uint2 c1 = encode8(f1, s);
+        if (g_ok) {
+            uint8_t* dst = q + static_cast<size_t>(t) * k + static_cast<size_t>(g) * 128 + lane * 8;
+            st_stream8(dst, c0);
+            st_stream8(dst + 64, c1);
             if (lane == 0) {
                 if (s_row) s_row[static_cast<size_t>(t) * G + g] = s;
                 s_k[static_cast<size_t>(g) * mp + t] = s;
@@ -165,8 +203,9 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const uint16_t* __res
     for (int j = 0; j < 8; ++j) {
         const uint32_t c = threadIdx.x + 256u * j;
         const size_t off = static_cast<size_t>(bn * 128u + (c >> 4)) * k + bg * 128u + (c & 15u) * 8u;
-        widen8(ld_stream16(w + off), f[j]);
-        amax = fmaxf(amax, absmax8(f[j]));
+        const uint4 v = ld_stream16(w + off);
+        widen8(v, f[j]);
+        amax = fmaxf(amax, absmax8_bits(v));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
@@ -198,6 +237,42 @@ __global__ void convert_e4m3_kernel(const float* __restrict__ in, uint8_t* __res
     }
 }
 
+// Exhaustive check of the quantizers' division against IEEE division. CTA b
+// takes amax = the non-negative bf16 with bit pattern b (0 .. 0x7F7F, every
+// finite value), forms s = group_scale(amax) and, for every bf16 x with
+// |x| <= amax and both signs, compares the e4m3 code of div2_by_scale with
+// the code of __fdiv_rn(x, s), and the fp32 quotients themselves.
+// counts[0] += pairs checked, counts[1] += code mismatches,
+// counts[2] += fp32 quotient mismatches.
+__global__ void __launch_bounds__(256) check_division_kernel(unsigned long long* __restrict__ counts) {
+    const uint32_t a_bits = blockIdx.x;
+    const float amax = __uint_as_float(a_bits << 16);
+    const float s = group_scale(amax);
+    const float r = __frcp_rn(s);
+    unsigned long long pairs = 0, code_bad = 0, quot_bad = 0;
+    for (uint32_t xb = threadIdx.x; xb <= a_bits; xb += blockDim.x) {
+        const float xp = __uint_as_float(xb << 16);
+        const float2 xv = make_float2(xp, -xp);
+        const float2 qf = div2_by_scale(xv, s, r);
+        const float qa = __fdiv_rn(xv.x, s), qb = __fdiv_rn(xv.y, s);
+        const uint16_t c_fast = cvt_e4m3x2(qf.x, qf.y);
+        const uint16_t c_ieee = cvt_e4m3x2(qa, qb);
+        pairs += 2;
+        code_bad += ((c_fast & 0xFF) != (c_ieee & 0xFF)) + ((c_fast >> 8) != (c_ieee >> 8));
+        quot_bad += (__float_as_uint(qf.x) != __float_as_uint(qa)) + (__float_as_uint(qf.y) != __float_as_uint(qb));
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        pairs += __shfl_xor_sync(0xFFFFFFFFu, pairs, o);
+        code_bad += __shfl_xor_sync(0xFFFFFFFFu, code_bad, o);
+        quot_bad += __shfl_xor_sync(0xFFFFFFFFu, quot_bad, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+        atomicAdd(&counts[0], pairs);
+        atomicAdd(&counts[1], code_bad);
+        atomicAdd(&counts[2], quot_bad);
+    }
+}
+
 // ------------------------------------------------------------ launchers --
 
 cudaError_t launch_quant_act(const QuantLaunch& L, cudaStream_t stream) {
@@ -208,7 +283,7 @@ cudaError_t launch_quant_act(const QuantLaunch& L, cudaStream_t stream) {
                                                          L.s_row, L.s_k, L.m, L.k, L.mp);
     } else {
         dim3 grid((G + 7) / 8, (L.m + kMultiRowsPerCta - 1) / kMultiRowsPerCta);
-        quant_act_multi_kernel<kMultiRowsPerCta><<<grid, 128, 0, stream>>>(
+        quant_act_multi_kernel<kMultiRowsPerCta><<<grid, 64, 0, stream>>>(
             static_cast<const uint16_t*>(L.x), static_cast<uint8_t*>(L.q), L.s_row, L.s_k, L.m, L.k, L.mp);
     }
     note_launch();
@@ -220,6 +295,14 @@ cudaError_t launch_quant_weight(const void* w, void* wq, float* w_scale, uint32_
     dim3 grid(k / 128, n / 128);
     quant_weight_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(w), static_cast<uint8_t*>(wq),
                                                   w_scale, k);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_check_division(unsigned long long* counts, cudaStream_t stream) {
+    cudaError_t e = cudaMemsetAsync(counts, 0, 3 * sizeof(unsigned long long), stream);
+    if (e != cudaSuccess) return e;
+    check_division_kernel<<<0x7F80, 256, 0, stream>>>(counts);
     note_launch();
     return cudaGetLastError();
 }

@@ -85,17 +85,19 @@ typedef struct {
 
 /*
  * The smallest M at which a multi-group quantizer whose CTA covers
- * `groups_per_cta` K-groups of `rows_per_cta` tokens reaches
- * `min_ctas_per_sm * sm_count` CTAs at this K. Its grid is
+ * `groups_per_cta` K-groups of `rows_per_cta` tokens reaches the CTA floor
+ * ceil(min_ctas_per_sm * sm_count) at this K. Its grid is
  * ceil((K/128)/groups_per_cta) x ceil(M/rows_per_cta) CTAs; with
  * rows_per_cta = 1 this is the pages' formula ceil(floor / grid_y)
  * (P-FL, `fp8_quant_hopper_min_m` and the per-K table of the module header:
  * 132 SMs, 8 groups, 2 CTAs/SM gives 53/44/16 at K = 5120/6144/17408).
- * fp8q_quant_pick applies exactly this function. Pure host function.
- * Returns 0 when k < 128 or groups_per_cta or rows_per_cta is 0.
+ * fp8q_quant_pick applies exactly this function, with the floor measured for
+ * B200 (2/3 of a CTA per SM for this library's multi-group kernel). Pure host
+ * function. Returns 0 when k < 128, groups_per_cta or rows_per_cta is 0, or
+ * min_ctas_per_sm is negative or NaN.
  */
 uint32_t fp8q_quant_floor_min_m(uint32_t k, uint32_t sm_count, uint32_t groups_per_cta, uint32_t rows_per_cta,
-                                uint32_t min_ctas_per_sm);
+                                float min_ctas_per_sm);
 
 /*
  * Which quantizer variant runs for (m, k) on a device with `sm_count` SMs,
@@ -221,6 +223,19 @@ fp8q_status fp8q_linear_noalloc(const void *x, const void *wq, const float *w_sc
  * Errors: NULL, UNSUPPORTED_DEVICE, CUDA.
  */
 fp8q_status fp8q_convert_e4m3(const float *in, uint8_t *out, size_t count, void *stream);
+
+/*
+ * Exhaustive device check of the quantizers' division. The quantizers form
+ * x / s from the correctly rounded reciprocal of s and one remainder
+ * correction instead of a full IEEE division per element. This call runs,
+ * for every finite non-negative bf16 amax (s = max(amax, 1e-10f)/448) and
+ * every bf16 x with |x| <= amax (both signs), that division and the IEEE
+ * division, and compares the e4m3 codes and the fp32 quotients.
+ *   counts  device pointer to 3 uint64: [0] pairs checked (1065402240),
+ *           [1] code mismatches, [2] fp32 quotient mismatches.
+ * Errors: NULL, UNSUPPORTED_DEVICE, CUDA.
+ */
+fp8q_status fp8q_check_division(unsigned long long *counts, void *stream);
 
 /* Number of kernels this library has launched in this process. */
 uint64_t fp8q_launch_count(void);

@@ -158,6 +158,15 @@ def test_convert_matches_oracle_encoder_exhaustively():
     assert np.array_equal(got, oracle.e4m3_encode_array(extra))
 
 
+def test_division_exhaustive_against_ieee():
+    """The quantizers' reciprocal-plus-correction division gives the code of the
+    IEEE quotient for every (x, amax) pair of bf16 values with |x| <= amax."""
+    pairs, code_bad, quot_bad = api.check_division()
+    assert pairs == 0x7F80 * 0x7F81
+    assert code_bad == 0
+    print(f"division check: {pairs} pairs, {code_bad} code mismatches, {quot_bad} quotient mismatches")
+
+
 @pytest.mark.parametrize("n,k", [(512, 512), (256, 384), (6144, 5120), (5120, 17408)])
 def test_quant_weight_bitexact(n, k):
     wb, wq_o, ws_o = oracle_w(n, k, 1000 + n % 7)

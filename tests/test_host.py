@@ -11,6 +11,7 @@ import os
 import re
 import subprocess
 
+import numpy as np
 import pytest
 
 from conftest import ROOT, golden_rows
@@ -77,16 +78,28 @@ def test_floor_reproduces_the_sign_of_fifteen_arms():
 
 
 def test_floor_rows_per_cta_generalisation():
-    # min M with ceil(G/8) * ceil(M/rpc) >= floor, checked by brute force
+    # min M with ceil(G/8) * ceil(M/rpc) >= ceil(f * sms), checked by brute force
+    import math
     for k in [128, 512, 5120, 6144, 17408]:
         for sms in [1, 132, 148]:
             for rpc in [1, 2, 4]:
-                mm = api.quant_floor_min_m(k, sms, 8, rpc, 2)
-                gy = -(-(k // 128) // 8)
-                ok = [m for m in range(1, 5000) if gy * -(-m // rpc) >= 2 * sms]
-                assert mm == ok[0], (k, sms, rpc)
+                for f in [2.0, 2.0 / 3.0, 0.5, 1.0]:
+                    mm = api.quant_floor_min_m(k, sms, 8, rpc, f)
+                    gy = -(-(k // 128) // 8)
+                    floor = max(1, math.ceil(float(np.float32(f)) * sms - 1e-9))  # the ABI takes a float
+                    ok = [m for m in range(1, 5000) if gy * -(-m // rpc) >= floor]
+                    assert mm == ok[0], (k, sms, rpc, f)
     assert api.quant_floor_min_m(64, 148, 8, 1, 2) == 0
     assert api.quant_floor_min_m(5120, 148, 0, 1, 2) == 0
+    assert api.quant_floor_min_m(5120, 148, 8, 1, float("nan")) == 0
+
+
+def test_b200_floor_picks_the_faster_variant_at_decode_widths():
+    """On 148 SMs the pick sends each decode arm to the variant that measured
+    faster on B200 (fixture tests/golden/quant_arms_b200.txt)."""
+    for m, k, faster in golden_rows("quant_arms_b200.txt"):
+        p = api.quant_pick(int(m), int(k), 148)
+        assert p.variant == (api.MULTI if faster == "multi" else api.SINGLE), (m, k)
 
 
 def test_pick_keeps_kernel_and_grid_together():
@@ -94,17 +107,17 @@ def test_pick_keeps_kernel_and_grid_together():
         for k in [512, 5120, 6144, 17408]:
             auto = api.quant_pick(m, k, 148)
             g = k // 128
-            min_m = api.quant_floor_min_m(k, 148, 8, 2, 2)
+            min_m = api.quant_floor_min_m(k, 148, 8, 4, 2.0 / 3.0)
             assert auto.variant == (api.MULTI if m >= min_m else api.SINGLE)
             assert auto.forced == 0
-            assert auto.floor_ctas == 2 * 148
-            assert auto.multi_ctas == -(-g // 8) * -(-m // 2)
+            assert auto.floor_ctas == 99
+            assert auto.multi_ctas == -(-g // 8) * -(-m // 4)
             single = api.quant_pick(m, k, 148, api.SINGLE)
             assert single.variant == api.SINGLE and single.forced == 1
             assert single.grid_x == m * g and single.block_x == 16 and single.groups_per_cta == 1
             multi = api.quant_pick(m, k, 148, api.MULTI)
-            assert multi.variant == api.MULTI and multi.grid_x == multi.multi_ctas and multi.block_x == 128
-            assert multi.groups_per_cta == 16
+            assert multi.variant == api.MULTI and multi.grid_x == multi.multi_ctas and multi.block_x == 64
+            assert multi.groups_per_cta == 32
 
 
 def test_pick_argument_errors():
@@ -171,6 +184,7 @@ def test_gemm_and_linear_argument_errors():
     assert lib.fp8q_quant_weight(ODD, B, C, 256, 512, None) == 3
     assert lib.fp8q_convert_e4m3(None, B, 4, None) == 1
     assert lib.fp8q_convert_e4m3(A, B, 0, None) == 0
+    assert lib.fp8q_check_division(None, None) == 1
 
 
 def test_no_device_reports_cuda_error_not_crash():
