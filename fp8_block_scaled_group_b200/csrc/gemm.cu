@@ -14,17 +14,21 @@
 // one scalar per row and weight block: a_s[t][g] * w_s[c/128][g]. TMEM holds
 // two partial buffers, so the MMA of block g+1 overlaps the promotion of g.
 //
-// Persistent kernel, one CTA of 12 warps per SM, output tile 128 x 256:
-//   warp 0      TMA producer: A [128 rows x 128 B] and B [256 rows x 128 B]
-//               per K block into a 4-stage ring (128-byte swizzle), and the
-//               block's 128 activation scales (one K-major row slice) into
-//               an 8-slot scale ring that the promotion warps release
-//   warp 1      TMEM allocator and MMA issuer (one thread), M=128 N=256 K=32
+// Persistent kernel on CTA pairs (clusters of 2, one CTA per SM). A pair
+// owns a 256 x 256 output tile and issues M=256 N=256 MMAs across both SMs
+// (cta_group::2): each CTA stages its own 128 rows of A and its own 128 of
+// the 256 rows of B, so each SM's shared memory carries a third less traffic
+// per flop than a single-SM 128 x 256 tile. Per CTA, 12 warps:
+//   warp 0      TMA producer: A [128 x 128 B] and B [128 x 128 B] per K block
+//               into a 6-stage ring (128-byte swizzle), completion counted on
+//               the even CTA's barrier; plus the block's 128 activation
+//               scales (one K-major row slice) into an 8-slot local ring
+//   warp 1      TMEM allocation for the pair; in the even CTA, the MMA issuer
 //   warps 2-3   idle after set-up
 //   warps 4-11  promotion + epilogue. Warp w reads TMEM lanes 32*(w%4)..+31
-//               (tile rows) and column half (w-4)/4 (128 columns, one weight
-//               block), one row per thread, 128 fp32 accumulators each
-// Tiles are visited M-fastest so the CTAs running at one time share weight
+//               of its own CTA (its tile rows) and column half (w-4)/4 (128
+//               columns, one weight block), one row per thread
+// Tiles are visited M-fastest so the pairs running at one time share weight
 // tiles through L2. Rows past M and columns past N are zero-filled by TMA
 // and never stored.
 #include <cuda_bf16.h>
@@ -43,15 +47,17 @@ __device__ uint32_t g_device_error = 0;
 
 namespace {
 
-constexpr uint32_t BM = 128;
-constexpr uint32_t BN = 256;
+constexpr uint32_t BM = 128;       // rows per CTA
+constexpr uint32_t BM_PAIR = 256;  // rows per CTA pair (one MMA)
+constexpr uint32_t BN = 256;       // output columns per tile
+constexpr uint32_t BN_CTA = 128;   // rows of B staged by each CTA
 constexpr uint32_t BK = 128;
-constexpr uint32_t kStages = 4;
+constexpr uint32_t kStages = 6;
 constexpr uint32_t kScaleStages = 8;
 constexpr uint32_t kThreads = 384;
 constexpr uint32_t kEpiWarps = 8;
 constexpr uint32_t kTileBytesA = BM * BK;
-constexpr uint32_t kTileBytesB = BN * BK;
+constexpr uint32_t kTileBytesB = BN_CTA * BK;
 constexpr uint32_t kScaleBytes = BM * 4;
 constexpr uint32_t kTmemCols = 2 * BN;  // two partial buffers of BN fp32 columns
 // Register split: warpgroup 0 (producer, MMA, idle) gives registers to the
@@ -73,6 +79,7 @@ struct __align__(1024) GemmSmem {
     uint64_t tempty[2];
     uint64_t mma_done;
     uint32_t tmem_base;
+    uint32_t _pad;
     uint32_t abort;
     uint32_t consumed;  // K blocks whose TMA data the MMA thread has seen land
 };
@@ -87,11 +94,18 @@ struct Shape {
 __device__ __forceinline__ void tile_coords(const Shape& sh, uint32_t tile, uint32_t& m0, uint32_t& n0) {
     const uint32_t tm = tile % sh.num_m;
     const uint32_t tn = tile / sh.num_m;
-    m0 = tm * BM;
+    m0 = tm * BM_PAIR;
     n0 = tn * BN;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// Spin for about `cycles` SM clocks (bounded by construction).
+__device__ __forceinline__ void spin_cycles(long long cycles) {
+    const long long t0 = clock64();
+    while (clock64() - t0 < cycles) {
+    }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmS, const float* __restrict__ w_s,
                             uint16_t* __restrict__ y, const Shape sh) {
@@ -99,11 +113,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t warp = threadIdx.x >> 5;
     const uint32_t lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const uint32_t pair = blockIdx.x >> 1;
+    const uint32_t num_pairs = gridDim.x >> 1;
     volatile uint32_t* abort = &sm.abort;
 
     if (threadIdx.x == 0) {
         for (uint32_t s = 0; s < kStages; ++s) {
-            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.full[s], 2);  // one expect-tx arrival from each CTA of the pair
             mbar_init(&sm.empty[s], 1);
         }
         for (uint32_t s = 0; s < kScaleStages; ++s) {
@@ -112,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (uint32_t b = 0; b < 2; ++b) {
             mbar_init(&sm.tfull[b], 1);
-            mbar_init(&sm.tempty[b], kEpiWarps);
+            mbar_init(&sm.tempty[b], 2 * kEpiWarps);  // promotion warps of both CTAs
         }
         mbar_init(&sm.mma_done, 1);
         sm.abort = 0;
@@ -125,11 +142,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmS);
     }
     if (warp == 1) {
-        tmem_alloc(&sm.tmem_base, kTmemCols);
-        tmem_relinquish();
+        tmem_alloc_pair(&sm.tmem_base, kTmemCols);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();  // barriers of both CTAs initialised before any remote arrive
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const uint32_t G = sh.G;
@@ -141,9 +158,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (warp == 0 && lane == 0) {
             uint32_t it = 0;
             bool ok = true;
-            for (uint32_t tile = blockIdx.x; ok && tile < sh.num_tiles; tile += gridDim.x) {
+            for (uint32_t tile = pair; ok && tile < sh.num_tiles; tile += num_pairs) {
                 uint32_t m0, n0;
                 tile_coords(sh, tile, m0, n0);
+                const int32_t my_m = static_cast<int32_t>(m0 + rank * BM);
+                const int32_t my_n = static_cast<int32_t>(n0 + rank * BN_CTA);
                 for (uint32_t kb = 0; kb < G; ++kb, ++it) {
                     const uint32_t s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
@@ -154,18 +173,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(&sm.sfull[ss], kScaleBytes);
-                    tma_load_2d(sm.a_scale[ss], &tmS, &sm.sfull[ss], static_cast<int32_t>(m0), static_cast<int32_t>(kb));
-                    mbar_arrive_expect_tx(&sm.full[s], kTileBytesA + kTileBytesB);
-                    tma_load_2d(sm.a[s], &tmA, &sm.full[s], static_cast<int32_t>(kb * BK), static_cast<int32_t>(m0));
-                    tma_load_2d(sm.b[s], &tmB, &sm.full[s], static_cast<int32_t>(kb * BK), static_cast<int32_t>(n0));
+                    tma_load_2d(sm.a_scale[ss], &tmS, &sm.sfull[ss], my_m, static_cast<int32_t>(kb));
+                    const uint32_t full_even = mapa_shared(smem_addr(&sm.full[s]), 0);
+                    mbar_arrive_expect_tx_cluster(full_even, kTileBytesA + kTileBytesB);
+                    tma_load_2d_pair(sm.a[s], &tmA, full_even, static_cast<int32_t>(kb * BK), my_m);
+                    tma_load_2d_pair(sm.b[s], &tmB, full_even, static_cast<int32_t>(kb * BK), my_n);
                     issued = it + 1;
                 }
             }
-        } else if (warp == 1 && lane == 0) {
-            constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+        } else if (warp == 1 && lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = idesc_e4m3_f32(BM_PAIR, BN);
             uint32_t it = 0;
             bool ok = true;
-            for (uint32_t tile = blockIdx.x; ok && tile < sh.num_tiles; tile += gridDim.x) {
+            for (uint32_t tile = pair; ok && tile < sh.num_tiles; tile += num_pairs) {
                 for (uint32_t kb = 0; kb < G; ++kb, ++it) {
                     const uint32_t s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
@@ -186,13 +206,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t bd = smem_desc_k_sw128(smem_addr(sm.b[s]));
 #pragma unroll
                     for (uint32_t kk = 0; kk < BK / 32; ++kk)  // K = 32 bytes per MMA: +2 in the address field
-                        mma_f8f6f4(d, ad + 2u * kk, bd + 2u * kk, idesc, kk > 0 ? 1u : 0u);
-                    mma_commit(&sm.empty[s]);
-                    mma_commit(&sm.tfull[b]);
+                        mma_f8f6f4_pair(d, ad + 2u * kk, bd + 2u * kk, idesc, kk > 0 ? 1u : 0u);
+                    mma_commit_pair_multicast(&sm.empty[s], 0x3);
+                    mma_commit_pair_multicast(&sm.tfull[b], 0x3);
                 }
             }
             // Every MMA this thread issued has completed once mma_done fires.
-            mma_commit(&sm.mma_done);
+            mma_commit_pair(&sm.mma_done);
             volatile uint32_t never = 0;
             mbar_wait(&sm.mma_done, 0, &never);
         }
@@ -202,12 +222,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t half = (warp - 4u) >> 2;
         const uint32_t lane_off = (quad * 32u) << 16;
         const uint32_t r_local = quad * 32u + lane;
+        const uint32_t tempty_even[2] = {mapa_shared(smem_addr(&sm.tempty[0]), 0),
+                                         mapa_shared(smem_addr(&sm.tempty[1]), 0)};
         uint32_t it = 0;
         bool ok = true;
-        for (uint32_t tile = blockIdx.x; ok && tile < sh.num_tiles; tile += gridDim.x) {
+        for (uint32_t tile = pair; ok && tile < sh.num_tiles; tile += num_pairs) {
             uint32_t m0, n0;
             tile_coords(sh, tile, m0, n0);
-            const uint32_t row = m0 + r_local;
+            const uint32_t row = m0 + rank * BM + r_local;
             const bool row_ok = row < sh.M;
             const uint32_t col0 = n0 + half * 128u;
             const bool col_ok = col0 < sh.N;
@@ -247,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive(&sm.tempty[b]);
+                    mbar_arrive_cluster(tempty_even[b]);
                     mbar_arrive(&sm.sempty[ss]);
                 }
             }
@@ -268,27 +290,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // Teardown. On the normal path every TMA load was consumed and every MMA
-    // was waited for. After a timed-out wait, first let the copies this CTA
-    // started land (bounded), then free TMEM.
+    // completed before the promotion warps finished. After a timed-out wait
+    // (in either CTA) the loads this pair started may still be landing:
+    // the even CTA waits for the ones it can see, and both CTAs then give
+    // in-flight copies a bounded grace period before the pair synchronises
+    // and frees TMEM.
     tc_fence_before();
     __syncthreads();
     if (*abort) {
         volatile uint32_t never = 0;
         if (threadIdx.x == 0) atomicOr(&g_device_error, 1u);
         if (warp == 0 && lane == 0) {
-            for (uint32_t it = sm.consumed; it < issued; ++it)
-                mbar_wait(&sm.full[it % kStages], (it / kStages) & 1u, &never);
-            // Scale slices land on their own barriers; the last
-            // kScaleStages issued may still be in flight.
+            if (rank == 0)
+                for (uint32_t it = sm.consumed; it < issued; ++it)
+                    mbar_wait(&sm.full[it % kStages], (it / kStages) & 1u, &never);
             const uint32_t first = issued > kScaleStages ? issued - kScaleStages : 0u;
             for (uint32_t it = first; it < issued; ++it)
                 mbar_wait(&sm.sfull[it % kScaleStages], (it / kScaleStages) & 1u, &never);
+            spin_cycles(200000);
         }
         __syncthreads();
     }
+    cluster_sync_all();  // no remote arrive or pair MMA can still target this CTA
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc_pair(tmem, kTmemCols);
     }
 }
 
@@ -385,7 +411,7 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream) {
     const KernelSetup& ks = setup_for_device();
     if (ks.err != cudaSuccess) return ks.err;
     CUtensorMap ta, tb, ts;
-    if (!make_map_u8(&ta, L.q, L.k, L.m, BM) || !make_map_u8(&tb, L.wq, L.k, L.n, BN) ||
+    if (!make_map_u8(&ta, L.q, L.k, L.m, BM) || !make_map_u8(&tb, L.wq, L.k, L.n, BN_CTA) ||
         !make_map_scales(&ts, L.s_k, L.mp, L.k / BK))
         return cudaErrorInvalidValue;
     Shape sh;
@@ -393,9 +419,10 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream) {
     sh.N = L.n;
     sh.G = L.k / BK;
     sh.Mp = L.mp;
-    sh.num_m = (L.m + BM - 1) / BM;
+    sh.num_m = (L.m + BM_PAIR - 1) / BM_PAIR;
     sh.num_tiles = sh.num_m * ((L.n + BN - 1) / BN);
-    const uint32_t grid = sh.num_tiles < static_cast<uint32_t>(ks.sms) ? sh.num_tiles : static_cast<uint32_t>(ks.sms);
+    const uint32_t max_pairs = static_cast<uint32_t>(ks.sms) / 2;
+    const uint32_t grid = 2 * (sh.num_tiles < max_pairs ? sh.num_tiles : max_pairs);
     gemm_blockscaled_kernel<<<grid, kThreads, kSmemBytes, stream>>>(ta, tb, ts, L.w_scale,
                                                                     static_cast<uint16_t*>(L.y), sh);
     note_launch();
