@@ -34,6 +34,7 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "internal.h"
@@ -318,6 +319,257 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
 }
 
+// ------------------------------------------------------ decode widths --
+//
+// M <= 64 tokens: the weight is the big operand, so the MMA is swapped.
+// Each CTA multiplies a 128-row slice of W (the MMA's M) by all the tokens
+// (the MMA's N, NT = 32 or 64 wide) over one contiguous range of K blocks:
+//   D[n][t] = sum_j wq[n][128g+j] * q[t][128g+j]          (tcgen05, fp32, TMEM)
+//   acc[n][t] += (w_s[n/128][g] * a_s[t][g]) * D[n][t]     (promotion, fp32)
+// One promotion thread owns one weight row and its NT token accumulators.
+// With only N/128 weight slices (40-48 at the pages' decode shapes), K is
+// split S ways and the S CTAs of a slice form a thread-block cluster; each
+// parks its [NT x 128] fp32 partial in shared memory and the cluster sums
+// the S partials through distributed shared memory in a fixed order (the
+// result does not depend on timing), each CTA storing a share of the token
+// rows as bf16. CTA = 6 warps: warp 0 TMA producer (W [128 x 128 B], tokens
+// [NT x 128 B] and the block's NT token scales per stage, 4 stages, so two
+// CTAs fit per SM and the clusters of a call fit the GPU at once), warp 1
+// TMEM allocator and MMA issuer, warps 2-5 promotion (warp w reads TMEM
+// lanes 32*(w%4)..+31). A stage is freed after five arrivals: the MMA's
+// commit and the four promotion warps that read its token scales.
+
+constexpr uint32_t kDecStages = 4;
+constexpr uint32_t kDecBufs = 4;
+constexpr uint32_t kDecThreads = 192;
+constexpr uint32_t kDecEpiWarps = 4;
+constexpr uint32_t kDecMaxSplit = 8;
+constexpr uint32_t kDecMaxTokens = 64;
+
+template <uint32_t NT>
+struct __align__(1024) DecodeSmem {
+    uint8_t w[kDecStages][BM * BK];
+    uint8_t t[kDecStages][NT * BK];
+    float t_scale[kDecStages][NT];
+    uint64_t full[kDecStages];
+    uint64_t empty[kDecStages];
+    uint64_t tfull[kDecBufs];
+    uint64_t tempty[kDecBufs];
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    uint32_t abort;
+    uint32_t consumed;
+};
+
+template <uint32_t NT>
+constexpr size_t decode_smem_bytes() {
+    return sizeof(DecodeSmem<NT>) + 1024;
+}
+
+struct DecodeShape {
+    uint32_t M, N, G, split;
+};
+
+template <uint32_t NT>
+__device__ __forceinline__ void tmem_load_nt(uint32_t taddr, uint32_t (&r)[NT]);
+
+template <>
+__device__ __forceinline__ void tmem_load_nt<64>(uint32_t taddr, uint32_t (&r)[64]) {
+    tmem_load64(taddr, r);
+}
+
+template <>
+__device__ __forceinline__ void tmem_load_nt<32>(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile(
+        "tcgen05.wait::ld.sync.aligned;"
+        : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+          "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+          "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+          "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+        :
+        : "memory");
+}
+
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+    return v;
+}
+
+template <uint32_t NT>
+__global__ void __launch_bounds__(kDecThreads, 2)
+    gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmT,
+                       const __grid_constant__ CUtensorMap tmS, const float* __restrict__ w_s,
+                       uint16_t* __restrict__ y, const DecodeShape sh) {
+    extern __shared__ uint8_t smem_raw[];
+    using Smem = DecodeSmem<NT>;
+    Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr uint32_t kCols = kDecBufs * NT;  // 128 or 256 TMEM columns
+    const uint32_t warp = threadIdx.x >> 5;
+    const uint32_t lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();  // the cluster spans grid x: rank == K split
+    const uint32_t nb = blockIdx.y;           // weight block row
+    const uint32_t n0 = nb * BM;
+    const uint32_t G = sh.G;
+    const uint32_t kb0 = rank * G / sh.split;
+    const uint32_t nk = (rank + 1) * G / sh.split - kb0;
+    volatile uint32_t* abort = &sm.abort;
+
+    if (threadIdx.x == 0) {
+        for (uint32_t s = 0; s < kDecStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1 + kDecEpiWarps);
+        }
+        for (uint32_t b = 0; b < kDecBufs; ++b) {
+            mbar_init(&sm.tfull[b], 1);
+            mbar_init(&sm.tempty[b], kDecEpiWarps);
+        }
+        mbar_init(&sm.mma_done, 1);
+        sm.abort = 0;
+        sm.consumed = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmW);
+        tma_prefetch_desc(&tmT);
+        tma_prefetch_desc(&tmS);
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, kCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    uint32_t issued = 0;
+
+    float acc[NT];
+#pragma unroll
+    for (uint32_t i = 0; i < NT; ++i) acc[i] = 0.0f;
+    const uint32_t r_local = (warp & 3u) * 32u + lane;  // weight row within the slice
+
+    if (warp == 0) {
+        if (lane == 0) {
+            for (uint32_t it = 0; it < nk; ++it) {
+                const uint32_t kb = kb0 + it;
+                const uint32_t s = it % kDecStages;
+                const uint32_t ph = (it / kDecStages) & 1u;
+                if (!mbar_wait(&sm.empty[s], ph ^ 1u, abort)) break;
+                mbar_arrive_expect_tx(&sm.full[s], BM * BK + NT * BK + NT * 4);
+                tma_load_2d(sm.w[s], &tmW, &sm.full[s], static_cast<int32_t>(kb * BK), static_cast<int32_t>(n0));
+                tma_load_2d(sm.t[s], &tmT, &sm.full[s], static_cast<int32_t>(kb * BK), 0);
+                tma_load_2d(sm.t_scale[s], &tmS, &sm.full[s], 0, static_cast<int32_t>(kb));
+                issued = it + 1;
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_e4m3_f32(BM, NT);
+            for (uint32_t it = 0; it < nk; ++it) {
+                const uint32_t s = it % kDecStages;
+                const uint32_t ph = (it / kDecStages) & 1u;
+                const uint32_t b = it % kDecBufs;
+                const uint32_t tph = (it / kDecBufs) & 1u;
+                if (!mbar_wait(&sm.full[s], ph, abort)) break;
+                sm.consumed = it + 1;
+                if (!mbar_wait(&sm.tempty[b], tph ^ 1u, abort)) break;
+                tc_fence_after();
+                const uint32_t d = tmem + b * NT;
+                const uint64_t ad = smem_desc_k_sw128(smem_addr(sm.w[s]));
+                const uint64_t bd = smem_desc_k_sw128(smem_addr(sm.t[s]));
+#pragma unroll
+                for (uint32_t kk = 0; kk < BK / 32; ++kk)
+                    mma_f8f6f4(d, ad + 2u * kk, bd + 2u * kk, idesc, kk > 0 ? 1u : 0u);
+                mma_commit(&sm.empty[s]);
+                mma_commit(&sm.tfull[b]);
+            }
+            mma_commit(&sm.mma_done);
+            volatile uint32_t never = 0;
+            mbar_wait(&sm.mma_done, 0, &never);
+        }
+    } else {
+        const float* ws_row = w_s + static_cast<size_t>(nb) * G;
+        const uint32_t lane_off = ((warp & 3u) * 32u) << 16;
+        float w_next = nk > 0 ? __ldg(ws_row + kb0) : 0.0f;
+        for (uint32_t it = 0; it < nk; ++it) {
+            const uint32_t s = it % kDecStages;
+            const uint32_t b = it % kDecBufs;
+            const uint32_t tph = (it / kDecBufs) & 1u;
+            const float wsc = w_next;
+            if (it + 1 < nk) w_next = __ldg(ws_row + kb0 + it + 1);
+            const bool got = mbar_wait(&sm.tfull[b], tph, abort);
+            if (!__all_sync(0xFFFFFFFFu, got)) break;
+            tc_fence_after();
+            uint32_t v[NT];
+            tmem_load_nt<NT>(tmem + lane_off + b * NT, v);
+#pragma unroll
+            for (uint32_t i = 0; i < NT; ++i) acc[i] = fmaf(wsc * sm.t_scale[s][i], __uint_as_float(v[i]), acc[i]);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&sm.tempty[b]);
+                mbar_arrive(&sm.empty[s]);  // this warp is done with the stage's token scales
+            }
+        }
+    }
+
+    // After a timed-out wait, let the copies this CTA started land (bounded).
+    tc_fence_before();
+    __syncthreads();
+    if (*abort) {
+        volatile uint32_t never = 0;
+        if (threadIdx.x == 0) atomicOr(&g_device_error, 1u);
+        if (warp == 0 && lane == 0)
+            for (uint32_t it = sm.consumed; it < issued; ++it)
+                mbar_wait(&sm.full[it % kDecStages], (it / kDecStages) & 1u, &never);
+        __syncthreads();
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kCols);
+    }
+
+    // Split-K reduction across the cluster. The operand stages are idle now
+    // (every MMA and copy of this CTA finished), so the weight stages hold
+    // this CTA's partial, transposed: red[t][row] (consecutive threads write
+    // consecutive words).
+    float* red = reinterpret_cast<float*>(&sm.w[0][0]);
+    if (warp >= 2) {
+#pragma unroll
+        for (uint32_t i = 0; i < NT; ++i) red[i * BM + r_local] = acc[i];
+    }
+    cluster_sync_all();
+    if (threadIdx.x < BM && !*abort) {
+        const uint32_t j = threadIdx.x;
+        const uint32_t red_addr = smem_addr(red);
+        for (uint32_t t = rank; t < sh.M; t += sh.split) {
+            // Issue every peer's load before adding (independent remote
+            // reads in flight together), then sum in rank order.
+            float part[kDecMaxSplit];
+#pragma unroll
+            for (uint32_t p = 0; p < kDecMaxSplit; ++p)
+                part[p] = p < sh.split ? ld_shared_cluster_f32(mapa_shared(red_addr + (t * BM + j) * 4u, p)) : 0.0f;
+            float sum = 0.0f;
+#pragma unroll
+            for (uint32_t p = 0; p < kDecMaxSplit; ++p) sum += part[p];
+            __nv_bfloat16 h = __float2bfloat16_rn(sum);
+            y[static_cast<size_t>(t) * sh.N + n0 + j] = *reinterpret_cast<uint16_t*>(&h);
+        }
+    }
+    cluster_sync_all();  // peers' partials stay in place until every CTA has read them
+}
+
 // ------------------------------------------------------------ host side --
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -348,14 +600,14 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t ro
     return r == CUDA_SUCCESS;
 }
 
-// The K-major activation scales [G, Mp] fp32 read as [1 x 128] row slices
-// (128 tokens of one K group); tokens past Mp read as zero.
-bool make_map_scales(CUtensorMap* map, const float* base, uint64_t mp, uint64_t g) {
+// The K-major activation scales [G, Mp] fp32 read as [1 x box] row slices
+// (box tokens of one K group); tokens past Mp read as zero.
+bool make_map_scales_box(CUtensorMap* map, const float* base, uint64_t mp, uint64_t g, uint32_t box_tokens) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {mp, g};
     cuuint64_t strides[1] = {mp * sizeof(float)};
-    cuuint32_t box[2] = {BM, 1};
+    cuuint32_t box[2] = {box_tokens, 1};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
@@ -407,12 +659,75 @@ cudaError_t read_clear_device_error(uint32_t* code, cudaStream_t stream) {
     return e;
 }
 
+template <uint32_t NT>
+cudaError_t decode_smem_optin() {
+    static std::once_flag once;
+    static cudaError_t err = cudaSuccess;
+    std::call_once(once, [] {
+        err = cudaFuncSetAttribute(gemm_decode_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(decode_smem_bytes<NT>()));
+    });
+    return err;
+}
+
+// K split for `slices` weight slices of G K blocks: about 1.6 CTAs per SM
+// in total (the B200 sweep of splits 1..8 at N = 6144 and 5120 found its
+// best times there: 240 CTAs for 48 and for 40 slices), at most 8 and at
+// most G. FP8Q_DECODE_SPLIT=<n> overrides it.
+uint32_t decode_split(uint32_t slices, uint32_t G, int sms) {
+    static const int forced = [] {
+        const char* e = std::getenv("FP8Q_DECODE_SPLIT");
+        return e ? std::atoi(e) : 0;
+    }();
+    const uint32_t limit = kDecMaxSplit < G ? kDecMaxSplit : G;
+    if (forced > 0) return static_cast<uint32_t>(forced) < limit ? static_cast<uint32_t>(forced) : limit;
+    const uint32_t target = static_cast<uint32_t>(sms) * 8u / 5u;
+    uint32_t s = (target + slices / 2) / slices;
+    if (s < 1) s = 1;
+    return s < limit ? s : limit;
+}
+
+template <uint32_t NT>
+cudaError_t launch_decode(const GemmLaunch& L, int sms, cudaStream_t stream) {
+    const cudaError_t attr_err = decode_smem_optin<NT>();
+    if (attr_err != cudaSuccess) return attr_err;
+    CUtensorMap tw, tt, ts;
+    if (!make_map_u8(&tw, L.wq, L.k, L.n, BM) || !make_map_u8(&tt, L.q, L.k, L.m, NT) ||
+        !make_map_scales_box(&ts, L.s_k, L.mp, L.k / BK, NT))
+        return cudaErrorInvalidValue;
+    DecodeShape sh;
+    sh.M = L.m;
+    sh.N = L.n;
+    sh.G = L.k / BK;
+    const uint32_t slices = L.n / BM;
+    const uint32_t split = decode_split(slices, sh.G, sms);
+    sh.split = split;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(split, slices, 1);
+    cfg.blockDim = dim3(kDecThreads, 1, 1);
+    cfg.dynamicSmemBytes = decode_smem_bytes<NT>();
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_decode_kernel<NT>, tw, tt, ts, L.w_scale,
+                                       static_cast<uint16_t*>(L.y), sh);
+    note_launch();
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream) {
     const KernelSetup& ks = setup_for_device();
     if (ks.err != cudaSuccess) return ks.err;
+    if (L.m <= 32) return launch_decode<32>(L, ks.sms, stream);
+    if (L.m <= kDecMaxTokens) return launch_decode<64>(L, ks.sms, stream);
     CUtensorMap ta, tb, ts;
     if (!make_map_u8(&ta, L.q, L.k, L.m, BM) || !make_map_u8(&tb, L.wq, L.k, L.n, BN_CTA) ||
-        !make_map_scales(&ts, L.s_k, L.mp, L.k / BK))
+        !make_map_scales_box(&ts, L.s_k, L.mp, L.k / BK, BM))
         return cudaErrorInvalidValue;
     Shape sh;
     sh.M = L.m;
