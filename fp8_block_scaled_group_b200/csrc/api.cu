@@ -233,7 +233,7 @@ fp8q_status fp8q_gemm_blockscaled(const void* q, const float* s_kmajor, const vo
     if (m == 0) return FP8Q_OK;
     DeviceInfo dev;
     if ((st = current_device(&dev)) != FP8Q_OK) return st;
-    GemmLaunch L{q, s_kmajor, wq, w_scale, y, m, n, k, fp8q_m_pad(m)};
+    GemmLaunch L{q, s_kmajor, wq, w_scale, y, m, n, k, fp8q_m_pad(m), false};
     return from_cuda(launch_gemm(L, static_cast<cudaStream_t>(stream)));
 }
 
@@ -260,7 +260,11 @@ fp8q_status fp8q_linear(const void* x, const void* wq, const float* w_scale, voi
     if ((st = check_gemm_args(ws, s_k, wq, w_scale, y, m, n, k)) != FP8Q_OK) return st;
     if (m == 0) return FP8Q_OK;
     if ((st = fp8q_quant_act(x, ws, nullptr, s_k, m, k, stream)) != FP8Q_OK) return st;
-    return fp8q_gemm_blockscaled(ws, s_k, wq, w_scale, y, m, n, k, stream);
+    // The GEMM is the quantizer's programmatic dependent: its set-up (barriers,
+    // TMEM, descriptor prefetch) overlaps the quantizer, and its producer waits
+    // for the quantizer's grid before the first load.
+    GemmLaunch L{ws, s_k, wq, w_scale, y, m, n, k, fp8q_m_pad(m), true};
+    return from_cuda(launch_gemm(L, static_cast<cudaStream_t>(stream)));
 }
 
 fp8q_status fp8q_convert_e4m3(const float* in, uint8_t* out, size_t count, void* stream) {

@@ -157,6 +157,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (warp < 4) {
         regs_dec<kRegsLow>();
         if (warp == 0 && lane == 0) {
+            // Set-up above overlaps the producing kernel (quantizer) when
+            // launched as its dependent; its outputs are read from here on.
+            grid_dependency_wait();
             uint32_t it = 0;
             bool ok = true;
             for (uint32_t tile = pair; ok && tile < sh.num_tiles; tile += num_pairs) {
@@ -461,6 +464,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 
     if (warp == 0) {
         if (lane == 0) {
+            grid_dependency_wait();
             for (uint32_t it = 0; it < nk; ++it) {
                 const uint32_t kb = kb0 + it;
                 const uint32_t s = it % kDecStages;
@@ -707,13 +711,15 @@ cudaError_t launch_decode(const GemmLaunch& L, int sms, cudaStream_t stream) {
     cfg.blockDim = dim3(kDecThreads, 1, 1);
     cfg.dynamicSmemBytes = decode_smem_bytes<NT>();
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = split;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = L.pdl ? 2 : 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_decode_kernel<NT>, tw, tt, ts, L.w_scale,
                                        static_cast<uint16_t*>(L.y), sh);
     note_launch();
@@ -738,10 +744,20 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream) {
     sh.num_tiles = sh.num_m * ((L.n + BN - 1) / BN);
     const uint32_t max_pairs = static_cast<uint32_t>(ks.sms) / 2;
     const uint32_t grid = 2 * (sh.num_tiles < max_pairs ? sh.num_tiles : max_pairs);
-    gemm_blockscaled_kernel<<<grid, kThreads, kSmemBytes, stream>>>(ta, tb, ts, L.w_scale,
-                                                                    static_cast<uint16_t*>(L.y), sh);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = L.pdl ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel, ta, tb, ts, L.w_scale,
+                                       static_cast<uint16_t*>(L.y), sh);
     note_launch();
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace fp8q

@@ -42,6 +42,7 @@ struct GemmLaunch {
     const float* w_scale;
     void* y;
     uint32_t m, n, k, mp;
+    bool pdl;  // launched as the programmatic dependent of the kernel before it
 };
 
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream);
