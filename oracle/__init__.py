@@ -2,7 +2,9 @@
 
 A ctypes wrapper around ``fp8q_oracle.c``: the plain, slow CPU restatement of
 per-token-group FP8 activation quantization, 128x128 block weight
-quantization and the float64 dequantized GEMM reference (pages
+quantization, the float64 dequantized GEMM reference, and the dense FFN built
+from them: SiLU(gate) * up rounded to bf16 and quantized again for the down
+projection (pages
 "spark_model/layers/ops/dispatch_proj.rs" and
 "spark_model/layers/ops/fp8_act_quant_floor.rs").
 
@@ -70,6 +72,14 @@ def _load():
         lib.oracle_gemm_ref_rows.restype = None
         lib.oracle_check_tolerance.argtypes = [P, P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_double)]
         lib.oracle_check_tolerance.restype = ctypes.c_size_t
+        lib.oracle_silu_mul_bf16.argtypes = [ctypes.c_uint16, ctypes.c_uint16]
+        lib.oracle_silu_mul_bf16.restype = ctypes.c_uint16
+        lib.oracle_silu_mul_bf16_array.argtypes = [P, P, ctypes.c_size_t, P]
+        lib.oracle_silu_mul_bf16_array.restype = None
+        lib.oracle_round_bf16_array.argtypes = [P, ctypes.c_size_t, P]
+        lib.oracle_round_bf16_array.restype = None
+        lib.oracle_silu_mul_quant.argtypes = [P, P, ctypes.c_size_t, U32, U32, P, P, P]
+        lib.oracle_silu_mul_quant.restype = ctypes.c_int
         _lib = lib
         return lib
 
@@ -178,3 +188,60 @@ def check_tolerance(y_bf16: np.ndarray, ref: np.ndarray):
     worst = ctypes.c_double(0.0)
     bad = _load().oracle_check_tolerance(_ptr(y), _ptr(r), y.size, ctypes.byref(worst))
     return int(bad), float(worst.value)
+
+
+# ------------------------------------------------------------ dense FFN --
+
+def silu_mul_bf16(gate_bf16: np.ndarray, up_bf16: np.ndarray) -> np.ndarray:
+    """h = bf16_rne(silu(gate) * up), elementwise over bf16 bit arrays."""
+    g = np.ascontiguousarray(gate_bf16, dtype=np.uint16)
+    u = np.ascontiguousarray(up_bf16, dtype=np.uint16)
+    assert g.shape == u.shape
+    h = np.empty(g.shape, np.uint16)
+    _load().oracle_silu_mul_bf16_array(_ptr(g), _ptr(u), g.size, _ptr(h))
+    return h
+
+
+def round_bf16(v: np.ndarray) -> np.ndarray:
+    """float64 -> bf16 bits, round to nearest, ties to even."""
+    a = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty(a.shape, np.uint16)
+    _load().oracle_round_bf16_array(_ptr(a), a.size, _ptr(out))
+    return out
+
+
+def silu_mul_quant(gate_bf16: np.ndarray, up_bf16: np.ndarray):
+    """bf16 bits gate, up [M, I] -> quant_act(silu(gate) * up) as
+    (q [M,I] u8, s_row [M,I/128] f32, s_kmajor [I/128, ceil16(M)] f32)."""
+    g = np.ascontiguousarray(gate_bf16, dtype=np.uint16)
+    u = np.ascontiguousarray(up_bf16, dtype=np.uint16)
+    assert g.shape == u.shape and g.ndim == 2
+    m, i = g.shape
+    if i % GROUP:
+        raise ValueError("the intermediate width must be a multiple of 128")
+    q = np.empty((m, i), np.uint8)
+    s_row = np.empty((m, i // GROUP), np.float32)
+    s_k = np.empty((i // GROUP, m_pad(m)), np.float32)
+    rc = _load().oracle_silu_mul_quant(_ptr(g), _ptr(u), i, m, i, _ptr(q), _ptr(s_row), _ptr(s_k))
+    assert rc == 0
+    return q, s_row, s_k
+
+
+def ffn_ref(x_bf16: np.ndarray, wq_gate_up: np.ndarray, ws_gate_up: np.ndarray,
+            wq_down: np.ndarray, ws_down: np.ndarray, threads: int = 1) -> dict:
+    """The dense FFN, each stage by its definition:
+        q_x, s_x  = quant_act(x)                           (once, for both)
+        gate, up  = bf16(gemm_ref(q_x, W_gate)), bf16(gemm_ref(q_x, W_up))
+        q_h, s_h  = quant_act(bf16(silu(gate) * up))
+        y         = gemm_ref(q_h, W_down)                  (float64)
+    The gate and up weights are one [2I, D] matrix, gate rows first.
+    Returns every stage in a dict."""
+    q_x, s_x, _ = quant_act(x_bf16)
+    gu = gemm_ref(q_x, s_x, wq_gate_up, ws_gate_up, threads=threads)
+    i = wq_gate_up.shape[0] // 2
+    gate = round_bf16(gu[:, :i])
+    up = round_bf16(gu[:, i:])
+    q_h, s_h, s_h_k = silu_mul_quant(gate, up)
+    y = gemm_ref(q_h, s_h, wq_down, ws_down, threads=threads)
+    return {"q_x": q_x, "s_x": s_x, "gate": gate, "up": up,
+            "q_h": q_h, "s_h": s_h, "s_h_kmajor": s_h_k, "y": y}

@@ -314,3 +314,146 @@ void oracle_e4m3_encode_array(const float *t, size_t count, uint8_t *out)
     for (i = 0; i < count; i++)
         out[i] = oracle_e4m3_encode(t[i]);
 }
+
+/* ------------------------------------------- dense FFN: SiLU(gate) * up -- */
+
+/*
+ * The dense FFN of dispatch_proj.rs (doc of `cublas_fp8_proj_prequant`)
+ * quantizes its input once for the gate and up projections, then quantizes
+ * "the post-SiLU intermediate" once more for the down projection. The pages
+ * print neither that activation nor its precision; the reading taken here:
+ *   gate, up  the bf16 outputs of the two projections
+ *   h         = bf16_rne( silu(gate) * up ),  silu(z) = z / (1 + e^-z),
+ *             the real value rounded once to bf16 (the quantizer's input
+ *             type), so that the definition does not depend on how an
+ *             exponential is approximated.
+ * Zero results keep the sign of gate*up (silu(z) has the sign of z).
+ */
+
+#if !defined(LDBL_MANT_DIG) || LDBL_MANT_DIG < 64
+#error "the SiLU oracle needs an extended long double (64-bit significand)"
+#endif
+
+/* bf16 bits of a finite, nonzero long double magnitude a, rounded to the
+   nearest bf16 (8-bit significand, binary32 exponent range), ties to even
+   unless tie_down is set, in which case a tie goes to the smaller value.
+   Overflow gives infinity (0x7F80). */
+static uint16_t bf16_magnitude_bits(long double a, int tie_down)
+{
+    int e;
+    long double q, fl, frac, n;
+    long double quantum;
+    uint32_t code;
+    if (a < ldexpl(1.0L, -126)) {
+        quantum = ldexpl(1.0L, -133);        /* subnormal spacing */
+    } else {
+        (void)frexpl(a, &e);                 /* a = f * 2^e, f in [0.5, 1) */
+        quantum = ldexpl(1.0L, e - 1 - 7);   /* 7 fraction bits below the leading one */
+    }
+    q = a / quantum;                         /* exact: scaling by a power of two */
+    fl = floorl(q);
+    frac = q - fl;
+    if (frac > 0.5L)
+        n = fl + 1.0L;
+    else if (frac < 0.5L)
+        n = fl;
+    else if (tie_down)
+        n = fl;
+    else
+        n = (fmodl(fl, 2.0L) == 0.0L) ? fl : fl + 1.0L;
+    a = n * quantum;                         /* the rounded magnitude, exact */
+    if (a >= ldexpl(1.0L, 128))
+        return 0x7F80;
+    {
+        float f = (float)a;                  /* exact: a is a bf16 value */
+        uint32_t u;
+        memcpy(&u, &f, sizeof u);
+        code = u >> 16;
+    }
+    return (uint16_t)code;
+}
+
+/*
+ * h = bf16_rne(silu(g) * u) for bf16 inputs g, u (bit patterns).
+ * P = g*u is exact in long double (two 8-bit significands). For g <= 32
+ * the value P / (1 + e^-g) is formed in long double (64-bit significand):
+ * its relative error is a few 2^-64, far below the bf16 rounding step, and
+ * since e^-g is transcendental for g != 0 the real value is never exactly a
+ * rounding tie. For g > 32 the factor 1/(1+e^-g) differs from 1 by less
+ * than 2^-46, while P (16 significant bits) either sits exactly on a bf16
+ * tie or lies at least 2^-17 |P| away from one; so the result is P rounded
+ * to bf16, except that an exact tie goes toward zero, because
+ * silu(g) < g for every g > 0.
+ */
+uint16_t oracle_silu_mul_bf16(uint16_t g_bits, uint16_t u_bits)
+{
+    float gf = oracle_bf16_to_f32(g_bits);
+    float uf = oracle_bf16_to_f32(u_bits);
+    long double g = (long double)gf, u = (long double)uf;
+    long double p = g * u;
+    uint16_t sign = (uint16_t)((g_bits ^ u_bits) & 0x8000u);
+    long double v;
+    if (p == 0.0L)
+        return sign;
+    if (g > 32.0L)
+        return (uint16_t)(sign | bf16_magnitude_bits(fabsl(p), 1));
+    v = p / (1.0L + expl(-g));
+    return (uint16_t)(sign | bf16_magnitude_bits(fabsl(v), 0));
+}
+
+/* Round each float64 value to bf16 bits, nearest, ties to even (the
+   projections' bf16 outputs in the FFN reference). Signed zeros kept. */
+void oracle_round_bf16_array(const double *v, size_t count, uint16_t *out)
+{
+    size_t i;
+    for (i = 0; i < count; i++) {
+        uint16_t sign = signbit(v[i]) ? 0x8000u : 0u;
+        out[i] = v[i] == 0.0 ? sign : (uint16_t)(sign | bf16_magnitude_bits(fabsl((long double)v[i]), 0));
+    }
+}
+
+/*
+ * SiLU-and-multiply followed by the per-token group quantization of the
+ * result, as the FFN feeds its down projection:
+ *   gate, up  bf16 bits; row t of gate starts at gate + t*ld, likewise up
+ *   h[t][j]   = oracle_silu_mul_bf16(gate[t][j], up[t][j]),  j < i
+ *   q, s_row, s_kmaj exactly as oracle_quant_act over h ([m, i])
+ * Returns 0, or -1 if i is not a multiple of 128.
+ */
+int oracle_silu_mul_quant(const uint16_t *gate, const uint16_t *up, size_t ld,
+                          uint32_t m, uint32_t i, uint8_t *q, float *s_row, float *s_kmaj)
+{
+    uint32_t G, mp, t, g, j;
+    float buf[GROUP];
+    if (i % GROUP != 0)
+        return -1;
+    G = i / GROUP;
+    mp = oracle_m_pad(m);
+    for (t = 0; t < m; t++) {
+        for (g = 0; g < G; g++) {
+            float s;
+            for (j = 0; j < GROUP; j++) {
+                size_t c = (size_t)g * GROUP + j;
+                buf[j] = oracle_bf16_to_f32(oracle_silu_mul_bf16(gate[(size_t)t * ld + c], up[(size_t)t * ld + c]));
+            }
+            s = quantize_group(buf, 1, GROUP, q + (size_t)t * i + (size_t)g * GROUP, 1);
+            if (s_row)
+                s_row[(size_t)t * G + g] = s;
+            if (s_kmaj)
+                s_kmaj[(size_t)g * mp + t] = s;
+        }
+    }
+    if (s_kmaj)
+        for (g = 0; g < G; g++)
+            for (t = m; t < mp; t++)
+                s_kmaj[(size_t)g * mp + t] = 0.0f;
+    return 0;
+}
+
+/* h for `count` (gate, up) pairs (sweeps). */
+void oracle_silu_mul_bf16_array(const uint16_t *g, const uint16_t *u, size_t count, uint16_t *h)
+{
+    size_t i;
+    for (i = 0; i < count; i++)
+        h[i] = oracle_silu_mul_bf16(g[i], u[i]);
+}
