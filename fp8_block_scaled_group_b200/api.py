@@ -124,6 +124,89 @@ def linear(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor, workspace: 
     return y
 
 
+def silu_mul_quant(gate: torch.Tensor, up: torch.Tensor, row_major: bool = True, out=None, stream=None):
+    """gate, up bf16 [M, I] (rows may be strided, e.g. the two halves of a
+    [M, 2I] buffer) -> quant_act(bf16(silu(gate) * up)) as
+    (q uint8 [M, I], s_row fp32 [M, I/128] or None, s_kmajor fp32 [I/128, ceil16(M)])."""
+    if gate.shape != up.shape or gate.dim() != 2:
+        raise ValueError("gate and up must be 2-D with the same shape")
+    m, i = gate.shape
+    for name, t in (("gate", gate), ("up", up)):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or t.stride(1) != 1:
+            raise ValueError(f"{name} must be a bf16 CUDA tensor with unit column stride")
+    ld = gate.stride(0) if m > 1 else i
+    if m > 1 and up.stride(0) != ld:
+        raise ValueError("gate and up must share one row stride")
+    g, mp = i // GROUP, m_pad(m)
+    if out is None:
+        q = torch.empty((m, i), dtype=torch.uint8, device=gate.device)
+        s_row = torch.empty((m, g), dtype=torch.float32, device=gate.device) if row_major else None
+        s_k = torch.empty((g, mp), dtype=torch.float32, device=gate.device)
+    else:
+        q, s_row, s_k = out
+    _lib.check(_lib.load().fp8q_silu_mul_quant(_p(gate), _p(up), ld, _p(q), _p(s_row), _p(s_k), m, i,
+                                                _stream(stream)), "fp8q_silu_mul_quant")
+    return q, s_row, s_k
+
+
+def ffn_workspace_layout(m: int, d: int, i: int) -> list[int]:
+    """Byte offsets of q_x, s_x, gate|up, q_h, s_h in the FFN workspace, then its size."""
+    off = (_lib.SZ * 6)()
+    _lib.check(_lib.load().fp8q_ffn_workspace_layout(m, d, i, off), "fp8q_ffn_workspace_layout")
+    return [int(v) for v in off]
+
+
+def ffn(x: torch.Tensor, wq_gate_up: torch.Tensor, ws_gate_up: torch.Tensor, wq_down: torch.Tensor,
+        ws_down: torch.Tensor, workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
+        stream=None) -> torch.Tensor:
+    """Dense FFN: x bf16 [M, D] -> y bf16 [M, D] with y = down(silu(gate(x)) * up(x)), x quantized once.
+    wq_gate_up uint8 [2I, D] (gate rows first), ws_gate_up fp32 [2I/128, D/128],
+    wq_down uint8 [D, I], ws_down fp32 [D/128, I/128]."""
+    m, d = x.shape
+    i = wq_gate_up.shape[0] // 2
+    _need(x, torch.bfloat16, (m, d), "x")
+    _need(wq_gate_up, torch.uint8, (2 * i, d), "wq_gate_up")
+    _need(ws_gate_up, torch.float32, (2 * i // GROUP, d // GROUP), "ws_gate_up")
+    _need(wq_down, torch.uint8, (d, i), "wq_down")
+    _need(ws_down, torch.float32, (d // GROUP, i // GROUP), "ws_down")
+    need = ffn_workspace_layout(m, d, i)[5]
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    y = torch.empty((m, d), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _need(y, torch.bfloat16, (m, d), "y")
+    _lib.check(_lib.load().fp8q_ffn(_p(x), _p(wq_gate_up), _p(ws_gate_up), _p(wq_down), _p(ws_down), _p(y),
+                                     _p(workspace), workspace.numel(), m, d, i, _stream(stream)), "fp8q_ffn")
+    return y
+
+
+def ffn_intermediates(workspace: torch.Tensor, m: int, d: int, i: int) -> dict:
+    """Views of the FFN's intermediates inside its workspace (after the call has run)."""
+    off = ffn_workspace_layout(m, d, i)
+    mp = m_pad(m)
+
+    def view(k, dtype, shape):
+        n = 1
+        for v in shape:
+            n *= v
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        return workspace[off[k]:off[k] + nbytes].view(dtype).view(*shape)
+
+    return {"q_x": view(0, torch.uint8, (m, d)), "s_x_kmajor": view(1, torch.float32, (d // GROUP, mp)),
+            "gate_up": view(2, torch.bfloat16, (m, 2 * i)), "q_h": view(3, torch.uint8, (m, i)),
+            "s_h_kmajor": view(4, torch.float32, (i // GROUP, mp))}
+
+
+def check_silu_mul(stream=None) -> tuple[int, int, int, float]:
+    """Exhaustive check of SiLU(gate)*up's fp32 path against its fp64 path; returns
+    (pairs, pairs on the fp32 path, of those the mismatches, worst fp32 error in ulps)."""
+    counts = torch.zeros(3, dtype=torch.int64, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _lib.check(_lib.load().fp8q_check_silu_mul(_p(counts), _p(err), _stream(stream)), "fp8q_check_silu_mul")
+    a, b, c = counts.cpu().tolist()
+    worst = float(err.cpu().view(torch.float32).item())
+    return int(a), int(b), int(c), worst
+
+
 def convert_e4m3(t: torch.Tensor, stream=None) -> torch.Tensor:
     """fp32 CUDA tensor -> uint8 e4m3 codes with the quantizers' conversion."""
     if not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():

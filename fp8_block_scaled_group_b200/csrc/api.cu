@@ -267,6 +267,88 @@ fp8q_status fp8q_linear(const void* x, const void* wq, const float* w_scale, voi
     return from_cuda(launch_gemm(L, static_cast<cudaStream_t>(stream)));
 }
 
+fp8q_status fp8q_silu_mul_quant(const void* gate, const void* up, uint32_t ld, void* q, float* s_row,
+                                float* s_kmajor, uint32_t m, uint32_t i, void* stream) {
+    if (i == 0 || i % kGroup || ld < i || ld % 8) return FP8Q_ERR_SHAPE;
+    if (m == 0) return FP8Q_OK;
+    if (!gate || !up || !q || !s_kmajor) return FP8Q_ERR_NULL;
+    if (static_cast<uint64_t>(m) * ld >= (1ull << 31)) return FP8Q_ERR_SHAPE;
+    if (!aligned16(gate) || !aligned16(up) || !aligned16(q) || !aligned16(s_kmajor) ||
+        (s_row && !aligned16(s_row)))
+        return FP8Q_ERR_ALIGN;
+    DeviceInfo dev;
+    fp8q_status st = current_device(&dev);
+    if (st != FP8Q_OK) return st;
+    SiluLaunch L{gate, up, ld, q, s_row, s_kmajor, m, i, fp8q_m_pad(m)};
+    return from_cuda(launch_silu_mul_quant(L, false, static_cast<cudaStream_t>(stream)));
+}
+
+fp8q_status fp8q_ffn_workspace_layout(uint32_t m, uint32_t d, uint32_t i, size_t* offsets) {
+    if (!offsets) return FP8Q_ERR_NULL;
+    if (d == 0 || d % kGroup || i == 0 || i % kGroup) return FP8Q_ERR_SHAPE;
+    const size_t mp = fp8q_m_pad(m);
+    size_t off = 0;
+    offsets[0] = off;  // q_x      e4m3 [m, d]
+    off += round_up(static_cast<size_t>(m) * d, 256);
+    offsets[1] = off;  // s_x      fp32 [d/128, ceil16(m)]
+    off += round_up((d / kGroup) * mp * sizeof(float), 256);
+    offsets[2] = off;  // gate|up  bf16 [m, 2i]
+    off += round_up(static_cast<size_t>(m) * 2 * i * sizeof(uint16_t), 256);
+    offsets[3] = off;  // q_h      e4m3 [m, i]
+    off += round_up(static_cast<size_t>(m) * i, 256);
+    offsets[4] = off;  // s_h      fp32 [i/128, ceil16(m)]
+    off += round_up((i / kGroup) * mp * sizeof(float), 256);
+    offsets[5] = off;  // total
+    return FP8Q_OK;
+}
+
+size_t fp8q_ffn_workspace_bytes(uint32_t m, uint32_t d, uint32_t i) {
+    size_t off[6];
+    return fp8q_ffn_workspace_layout(m, d, i, off) == FP8Q_OK ? off[5] : 0;
+}
+
+fp8q_status fp8q_ffn(const void* x, const void* w_gate_up, const float* w_gate_up_scale, const void* w_down,
+                     const float* w_down_scale, void* y, void* workspace, size_t workspace_bytes, uint32_t m,
+                     uint32_t d, uint32_t i, void* stream) {
+    size_t off[6];
+    fp8q_status st = fp8q_ffn_workspace_layout(m, d, i, off);
+    if (st != FP8Q_OK) return st;
+    if (m == 0) return FP8Q_OK;
+    if (!x || !w_gate_up || !w_gate_up_scale || !w_down || !w_down_scale || !y || !workspace) return FP8Q_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < off[5]) return FP8Q_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    void* q_x = ws + off[0];
+    float* s_x = reinterpret_cast<float*>(ws + off[1]);
+    uint16_t* gu = reinterpret_cast<uint16_t*>(ws + off[2]);
+    void* q_h = ws + off[3];
+    float* s_h = reinterpret_cast<float*>(ws + off[4]);
+    if ((st = check_quant_args(x, q_x, nullptr, s_x, m, d)) != FP8Q_OK) return st;
+    if ((st = check_gemm_args(q_x, s_x, w_gate_up, w_gate_up_scale, gu, m, 2 * i, d)) != FP8Q_OK) return st;
+    if ((st = check_gemm_args(q_h, s_h, w_down, w_down_scale, y, m, d, i)) != FP8Q_OK) return st;
+    DeviceInfo dev;
+    if ((st = current_device(&dev)) != FP8Q_OK) return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const uint32_t mp = fp8q_m_pad(m);
+    // x is quantized once; gate and up come out of one GEMM over the stacked
+    // [2i, d] weight. Each later launch is the programmatic dependent of the
+    // one before it and waits on it before reading its output.
+    if ((st = fp8q_quant_act(x, q_x, nullptr, s_x, m, d, stream)) != FP8Q_OK) return st;
+    GemmLaunch gate_up{q_x, s_x, w_gate_up, w_gate_up_scale, gu, m, 2 * i, d, mp, true};
+    if ((st = from_cuda(launch_gemm(gate_up, s))) != FP8Q_OK) return st;
+    SiluLaunch act{gu, gu + i, 2 * i, q_h, nullptr, s_h, m, i, mp};
+    if ((st = from_cuda(launch_silu_mul_quant(act, true, s))) != FP8Q_OK) return st;
+    GemmLaunch down{q_h, s_h, w_down, w_down_scale, y, m, d, i, mp, true};
+    return from_cuda(launch_gemm(down, s));
+}
+
+fp8q_status fp8q_check_silu_mul(unsigned long long* counts, uint32_t* max_err_bits, void* stream) {
+    if (!counts || !max_err_bits) return FP8Q_ERR_NULL;
+    DeviceInfo dev;
+    fp8q_status st = current_device(&dev);
+    if (st != FP8Q_OK) return st;
+    return from_cuda(launch_check_silu_mul(counts, max_err_bits, static_cast<cudaStream_t>(stream)));
+}
+
 fp8q_status fp8q_convert_e4m3(const float* in, uint8_t* out, size_t count, void* stream) {
     if (!in || !out) return FP8Q_ERR_NULL;
     if (count == 0) return FP8Q_OK;

@@ -47,6 +47,20 @@ struct GemmLaunch {
 
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream);
 
+// SiLU(gate) * up rounded to bf16, then quantized per 128-group of tokens.
+struct SiluLaunch {
+    const void* gate;
+    const void* up;
+    uint32_t ld;  // elements between consecutive rows of gate and of up
+    void* q;
+    float* s_row;
+    float* s_k;
+    uint32_t m, i, mp;
+};
+
+cudaError_t launch_silu_mul_quant(const SiluLaunch& L, bool pdl, cudaStream_t stream);
+cudaError_t launch_check_silu_mul(unsigned long long* counts, uint32_t* max_err_bits, cudaStream_t stream);
+
 cudaError_t read_clear_device_error(uint32_t* code, cudaStream_t stream);
 
 void note_launch();

@@ -22,107 +22,11 @@
 //           in flight.
 #include <cuda_bf16.h>
 
+#include "group_quant.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
 namespace fp8q {
-
-__device__ __forceinline__ uint4 ld_stream16(const void* p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
-
-__device__ __forceinline__ void st_stream8(void* p, uint2 v) {
-    asm volatile("st.global.cs.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
-}
-
-// 8 packed bf16 -> 8 fp32 (exact widening).
-__device__ __forceinline__ void widen8(const uint4 v, float (&f)[8]) {
-    f[0] = __uint_as_float(v.x << 16);
-    f[1] = __uint_as_float(v.x & 0xFFFF0000u);
-    f[2] = __uint_as_float(v.y << 16);
-    f[3] = __uint_as_float(v.y & 0xFFFF0000u);
-    f[4] = __uint_as_float(v.z << 16);
-    f[5] = __uint_as_float(v.z & 0xFFFF0000u);
-    f[6] = __uint_as_float(v.w << 16);
-    f[7] = __uint_as_float(v.w & 0xFFFF0000u);
-}
-
-// |x| maximum of 8 packed bf16, as fp32. With the sign bits cleared, finite
-// non-negative IEEE values order like their bit patterns, so the maximum is
-// taken on the integers, two 16-bit lanes at a time.
-__device__ __forceinline__ float absmax8_bits(const uint4 v) {
-    const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
-                                __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
-    const uint32_t hi = m >> 16, lo = m & 0xFFFFu;
-    return __uint_as_float((hi > lo ? hi : lo) << 16);
-}
-
-// The scale of a group with absolute maximum `amax`: one fp32 division.
-__device__ __forceinline__ float group_scale(float amax) {
-    return __fdiv_rn(fmaxf(amax, 1e-10f), 448.0f);
-}
-
-// x / s for a pair of values, rounded to nearest even, from the correctly
-// rounded reciprocal r = RN(1/s) and one remainder correction (Markstein's
-// division scheme, P. Markstein, IBM J. Res. Dev. 34(1), 1990):
-//   q0 = RN(x * r),  e = RN(x - q0 * s) (exact with a fused multiply-add),
-//   q  = RN(q0 + e * r).
-// The sign of x is put back at the end so that -0 stays -0. For every pair
-// (x, amax) of bf16 values with |x| <= amax, the code this gives equals the
-// code of the IEEE quotient: fp8q_check_division verifies it exhaustively on
-// the device.
-__device__ __forceinline__ float2 div2_by_scale(float2 x, float s, float r) {
-    const float2 q0 = __fmul2_rn(x, make_float2(r, r));
-    const float2 e = __ffma2_rn(make_float2(-q0.x, -q0.y), make_float2(s, s), x);
-    const float2 q = __ffma2_rn(e, make_float2(r, r), q0);
-    return make_float2(__uint_as_float(__float_as_uint(q.x) | (__float_as_uint(x.x) & 0x80000000u)),
-                       __uint_as_float(__float_as_uint(q.y) | (__float_as_uint(x.y) & 0x80000000u)));
-}
-
-// 8 values / s -> 8 codes packed little-endian.
-__device__ __forceinline__ uint2 encode8(const float (&f)[8], float s) {
-    const float r = __frcp_rn(s);
-    uint32_t c[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 q = div2_by_scale(make_float2(f[2 * i], f[2 * i + 1]), s, r);
-        c[i] = cvt_e4m3x2(q.x, q.y);
-    }
-    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
-}
-
-// Let a dependent kernel (the GEMM of a fused linear, launched with
-// programmatic stream serialization) start its set-up while this grid runs.
-// The dependent may launch once every CTA has either triggered or exited.
-// Measured on B200: when every CTA triggers, the GEMM launches as soon as
-// the last quantizer CTA has started, which takes ~0.7 us off a
-// decode-width linear; but on grids of about 2000 or more of these small
-// CTAs, triggering from all of them slows the quantizer itself by ~0.6 us.
-// So the single-group kernel triggers only on grids of at most 1024 CTAs,
-// and the multi-group kernel only from its last 2048 CTAs.
-constexpr uint32_t kSingleTriggerMaxGrid = 1024;
-constexpr uint32_t kMultiTriggerTail = 2048;
-
-__device__ __forceinline__ void trigger_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-// Zero the pad rows m..mp-1 of the K-major scales, spread over the grid.
-__device__ __forceinline__ void zero_kmajor_pad(float* __restrict__ s_k, uint32_t m, uint32_t mp, uint32_t G) {
-    const uint32_t pad = mp - m;
-    if (pad == 0) return;
-    const uint32_t nblk = gridDim.x * gridDim.y;
-    const uint32_t bid = blockIdx.y * gridDim.x + blockIdx.x;
-    const uint32_t total = pad * G;
-    for (uint32_t p = bid * blockDim.x + threadIdx.x; p < total; p += nblk * blockDim.x) {
-        const uint32_t g = p / pad;
-        s_k[static_cast<size_t>(g) * mp + m + (p - g * pad)] = 0.0f;
-    }
-}
 
 // SINGLE: blockDim 16, grid (G, M): CTA (g, t) quantizes group g of token t.
 __global__ void __launch_bounds__(16) quant_act_single_kernel(const uint16_t* __restrict__ x,

@@ -13,6 +13,13 @@ M in {16, 17, 25} and prefill widths M in {1168, 4576}, with K in
                    probability p, by a draw from N(0, sigma)  (outliers)
   W  bf16 [N, K]:  N(0, 0.02)
 
+The dense FFN (dispatch_proj.rs, doc of `cublas_fp8_proj_prequant`) is
+taken at hidden size D = 5120 and intermediate size I = 17408, the two
+projection shapes above (gate/up: N = 17408, K = 5120; down: N = 5120,
+K = 17408); its gate and up weights are one [2I, D] draw, gate rows first.
+For the SiLU-and-multiply step alone, gate and up are drawn like the
+projections' outputs: N(0, 3) (sqrt(5120) * 0.02 * rms(X) ~ 3), bf16.
+
 Generator: numpy PCG64 seeded with (1000 + config number, tag, M, K) so
 every shape has its own stream; fp32 draws are rounded to bf16 with
 round-to-nearest-even.
@@ -25,6 +32,8 @@ import numpy as np
 
 _TAG_X = 1
 _TAG_W = 2
+_TAG_GATE = 3
+_TAG_UP = 4
 
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -60,6 +69,13 @@ def weights(n: int, k: int, seed: int, sigma: float = 0.02) -> np.ndarray:
     rng = _rng(seed, _TAG_W, n, k)
     w = rng.standard_normal((n, k), dtype=np.float32) * np.float32(sigma)
     return f32_to_bf16_bits(w)
+
+
+def gate_up(m: int, i: int, seed: int, sigma: float = 3.0) -> tuple[np.ndarray, np.ndarray]:
+    """gate, up bf16 bits [m, i]: independent N(0, sigma) draws."""
+    g = _rng(seed, _TAG_GATE, m, i).standard_normal((m, i), dtype=np.float32) * np.float32(sigma)
+    u = _rng(seed, _TAG_UP, m, i).standard_normal((m, i), dtype=np.float32) * np.float32(sigma)
+    return f32_to_bf16_bits(g), f32_to_bf16_bits(u)
 
 
 @dataclass(frozen=True)
@@ -101,3 +117,28 @@ CONFIGS: dict[int, list[Workload]] = {
 
 def all_workloads() -> list[Workload]:
     return [w for n in sorted(CONFIGS) for w in CONFIGS[n]]
+
+
+@dataclass(frozen=True)
+class FfnWorkload:
+    """One dense-FFN shape: x [M, D] -> gate|up [M, 2I] -> h [M, I] -> y [M, D]."""
+    name: str
+    m: int
+    d: int
+    i: int
+    seed: int = 1100
+
+    def x(self) -> np.ndarray:
+        return activations(self.m, self.d, self.seed)
+
+    def w_gate_up(self) -> np.ndarray:
+        return weights(2 * self.i, self.d, self.seed)
+
+    def w_down(self) -> np.ndarray:
+        return weights(self.d, self.i, self.seed + 1)
+
+
+FFN_CONFIGS: list[FfnWorkload] = [
+    FfnWorkload("ffn_m25_d5120_i17408", 25, 5120, 17408),
+    FfnWorkload("ffn_m1168_d5120_i17408", 1168, 5120, 17408),
+]

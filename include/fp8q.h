@@ -15,7 +15,10 @@
  *   - the fused linear that runs both in one call (P-DP, `cublas_fp8_proj`);
  *   - the choice between the one-group-per-CTA and the multi-group-per-CTA
  *     quantizer by a CTA-count floor (P-FL, module header and
- *     `fp8_act_quant_hopper_reject`), re-derived for the device's SM count.
+ *     `fp8_act_quant_hopper_reject`), re-derived for the device's SM count;
+ *   - the dense FFN that quantizes its input once for the gate and up
+ *     projections and quantizes the post-SiLU intermediate once for the down
+ *     projection (P-DP, doc of `cublas_fp8_proj_prequant`).
  *
  * Conventions shared by every call:
  *   - Data pointers are DEVICE pointers owned by the caller, 16-byte aligned.
@@ -214,6 +217,62 @@ fp8q_status fp8q_linear(const void *x, const void *wq, const float *w_scale, voi
 fp8q_status fp8q_linear_noalloc(const void *x, const void *wq, const float *w_scale, void *y,
                                 uint32_t m, uint32_t n, uint32_t k, void *stream);
 
+/* --------------------------------------------------------- dense FFN ---- */
+
+/*
+ * SiLU(gate) * up, then the activation quantization of the result, as the
+ * dense FFN feeds its down projection (P-DP, doc of
+ * `cublas_fp8_proj_prequant`: "quantizes the post-SiLU intermediate once for
+ * `down`"). The pages do not print the activation; this library defines
+ *   h[t][j] = bf16_rne( silu(gate[t][j]) * up[t][j] ),
+ *   silu(z) = z / (1 + e^-z),
+ * the real value rounded once to bf16 (ties to even; a zero result carries
+ * the sign of gate*up), and then quantizes h exactly as fp8q_quant_act
+ * quantizes x: same group arithmetic, same codes, same two scale layouts.
+ *   gate, up   bf16, m rows of i values; row t starts at gate + t*ld
+ *              (likewise up), ld >= i and a multiple of 8 (inputs)
+ *   q          e4m3 [m, i]                       (output)
+ *   s_rowmajor fp32 [m, i/128] or NULL           (output)
+ *   s_kmajor   fp32 [i/128, ceil16(m)], pad rows zeroed (output, required)
+ * i must be a multiple of 128; m*ld below 2^31.
+ * Errors: NULL, ALIGN, SHAPE, UNSUPPORTED_DEVICE, CUDA.
+ */
+fp8q_status fp8q_silu_mul_quant(const void *gate, const void *up, uint32_t ld, void *q,
+                                float *s_rowmajor, float *s_kmajor,
+                                uint32_t m, uint32_t i, void *stream);
+
+/*
+ * Workspace of fp8q_ffn for (m, d, i): offsets[0..4] are the byte offsets
+ * of q_x e4m3 [m, d], s_x fp32 [d/128, ceil16(m)], gate|up bf16 [m, 2i]
+ * (row t: i gate values, then i up values), q_h e4m3 [m, i] and
+ * s_h fp32 [i/128, ceil16(m)], each 256-byte aligned; offsets[5] is the
+ * total size. Errors: NULL, SHAPE (d or i not a positive multiple of 128).
+ */
+fp8q_status fp8q_ffn_workspace_layout(uint32_t m, uint32_t d, uint32_t i, size_t *offsets);
+size_t fp8q_ffn_workspace_bytes(uint32_t m, uint32_t d, uint32_t i);
+
+/*
+ * Dense FFN with FP8 weights (P-DP, doc of `cublas_fp8_proj_prequant`):
+ *   q_x, s_x   = quant(x)                        once, for gate and up
+ *   [gate|up]  = gemm(q_x, w_gate_up)            one GEMM, N = 2i, bf16 out
+ *   q_h, s_h   = fp8q_silu_mul_quant(gate, up)
+ *   y          = gemm(q_h, w_down)               bf16 out
+ * Every intermediate stays in the workspace for inspection.
+ *   x               bf16 [m, d]                                  (input)
+ *   w_gate_up       e4m3 [2i, d]: rows 0..i-1 gate, i..2i-1 up    (input)
+ *   w_gate_up_scale fp32 [2i/128, d/128]                         (input)
+ *   w_down          e4m3 [d, i], w_down_scale fp32 [d/128, i/128] (inputs)
+ *   y               bf16 [m, d]                                  (output)
+ *   workspace       >= fp8q_ffn_workspace_bytes(m, d, i), 256-byte aligned
+ * d and i must be multiples of 128. The four kernels are chained on
+ * `stream`, each a programmatic dependent of the one before it.
+ * Errors: NULL, ALIGN, SHAPE, WORKSPACE, UNSUPPORTED_DEVICE, CUDA.
+ */
+fp8q_status fp8q_ffn(const void *x, const void *w_gate_up, const float *w_gate_up_scale,
+                     const void *w_down, const float *w_down_scale, void *y,
+                     void *workspace, size_t workspace_bytes,
+                     uint32_t m, uint32_t d, uint32_t i, void *stream);
+
 /* ------------------------------------------------------- diagnostics ---- */
 
 /*
@@ -236,6 +295,21 @@ fp8q_status fp8q_convert_e4m3(const float *in, uint8_t *out, size_t count, void 
  * Errors: NULL, UNSUPPORTED_DEVICE, CUDA.
  */
 fp8q_status fp8q_check_division(unsigned long long *counts, void *stream);
+
+/*
+ * Exhaustive device check of SiLU(gate) * up. fp8q_silu_mul_quant forms h
+ * in fp32 with the hardware exponential and reciprocal and falls back to an
+ * exact fp64 evaluation near bf16 rounding ties and outside the fp32 path's
+ * accurate range. This call runs both evaluations on every pair of finite
+ * bf16 (gate, up).
+ *   counts        device pointer to 3 uint64: [0] pairs (4261478400),
+ *                 [1] pairs where the fp32 path is taken, [2] of those, the
+ *                 pairs whose bf16 result differs from the fp64 path's
+ *   max_err_bits  device pointer to 1 uint32: the largest error of the fp32
+ *                 value, in fp32 ulps, as the bit pattern of an fp32 number
+ * Errors: NULL, UNSUPPORTED_DEVICE, CUDA.
+ */
+fp8q_status fp8q_check_silu_mul(unsigned long long *counts, uint32_t *max_err_bits, void *stream);
 
 /* Number of kernels this library has launched in this process. */
 uint64_t fp8q_launch_count(void);

@@ -187,6 +187,40 @@ def test_gemm_and_linear_argument_errors():
     assert lib.fp8q_check_division(None, None) == 1
 
 
+def test_silu_mul_quant_and_ffn_argument_errors():
+    lib = _lib.load()
+    # fp8q_silu_mul_quant(gate, up, ld, q, s_row, s_k, m, i, stream)
+    assert lib.fp8q_silu_mul_quant(None, None, 128, None, None, None, 0, 128, None) == 0
+    assert lib.fp8q_silu_mul_quant(A, B, 128, C, None, D, 1, 100, None) == 2
+    assert lib.fp8q_silu_mul_quant(A, B, 64, C, None, D, 1, 128, None) == 2    # ld < i
+    assert lib.fp8q_silu_mul_quant(A, B, 260, C, None, D, 1, 256, None) == 2   # ld not a multiple of 8
+    assert lib.fp8q_silu_mul_quant(A, B, 256, C, None, None, 1, 256, None) == 1
+    assert lib.fp8q_silu_mul_quant(ODD, B, 256, C, None, D, 1, 256, None) == 3
+    assert lib.fp8q_silu_mul_quant(A, B, 1 << 16, C, None, D, 1 << 15, 256, None) == 2
+    assert lib.fp8q_check_silu_mul(None, A, None) == 1
+    # fp8q_ffn(x, w_gu, s_gu, w_dn, s_dn, y, ws, ws_bytes, m, d, i, stream)
+    m, d, i = 17, 256, 384
+    need = lib.fp8q_ffn_workspace_bytes(m, d, i)
+    ws = ctypes.c_void_p(0x1000000)
+    assert lib.fp8q_ffn(None, None, None, None, None, None, None, 0, 0, d, i, None) == 0
+    assert lib.fp8q_ffn(A, B, C, D, E, A, ws, need, m, d, 100, None) == 2
+    assert lib.fp8q_ffn(A, B, C, D, E, None, ws, need, m, d, i, None) == 1
+    assert lib.fp8q_ffn(A, B, C, D, E, A, ws, need - 1, m, d, i, None) == 4
+    assert lib.fp8q_ffn(A, B, C, D, E, A, ctypes.c_void_p(0x1000010), need, m, d, i, None) == 4
+    assert lib.fp8q_ffn(A, B, C, D, ODD, A, ws, need, m, d, i, None) == 3
+
+
+def test_ffn_workspace_layout():
+    for m, d, i in [(1, 128, 128), (17, 256, 384), (25, 5120, 17408), (1168, 5120, 17408)]:
+        off = api.ffn_workspace_layout(m, d, i)
+        mp = api.m_pad(m)
+        sizes = [m * d, 4 * (d // 128) * mp, 2 * m * 2 * i, m * i, 4 * (i // 128) * mp]
+        for k in range(5):
+            assert off[k] % 256 == 0 and off[k + 1] >= off[k] + sizes[k]
+        assert api.ffn_workspace_layout(m, d, i)[5] == _lib.load().fp8q_ffn_workspace_bytes(m, d, i)
+    assert _lib.load().fp8q_ffn_workspace_bytes(1, 100, 128) == 0
+
+
 def test_no_device_reports_cuda_error_not_crash():
     """With valid arguments and no usable device, calls fail with a status."""
     import torch
