@@ -41,6 +41,13 @@ WORKLOADS = {
     "decode_m25_n6144_k5120": dict(m=25, n=6144, k=5120, p=0.01, sigma=20.0, number=2),
     "decode_m25_n5120_k17408": dict(m=25, n=5120, k=17408, p=0.01, sigma=20.0, number=3),
 }
+# The dense FFN built on the same kernels (x quantized once, one gate|up
+# GEMM, SiLU*up quantized for the down GEMM): D = 5120, I = 17408.
+FFN_WORKLOADS = {
+    "ffn_m1168_d5120_i17408": dict(m=1168, d=5120, i=17408, seed=1100),
+    "ffn_m25_d5120_i17408": dict(m=25, d=5120, i=17408, seed=1100),
+}
+FFN_METRIC = "dense FFN (FP8 block-scaled, x quantized once) TFLOP/s"
 DEFAULT_WORKLOAD = "prefill_m1168_n17408_k5120"
 N_SETS = 3
 
@@ -436,17 +443,201 @@ def ours_arm(args):
     return 0
 
 
+_FFN_ORACLE_W = {}
+
+
+def ffn_oracle_sample(wl: dict, threads: int):
+    """Time the oracle's FFN on a bounded sample of one step's token rows;
+    returns (TFLOP/s equivalent, rows, seconds). Weight preparation is not
+    part of the step and is done once."""
+    import oracle
+    from fp8_block_scaled_group_b200 import inputs
+    m, d, i = wl["m"], wl["d"], wl["i"]
+    xb = inputs.activations(m, d, wl["seed"])
+    key = (d, i, wl["seed"])
+    if key not in _FFN_ORACLE_W:
+        _FFN_ORACLE_W[key] = (*oracle.quant_weight(inputs.weights(2 * i, d, wl["seed"])),
+                              *oracle.quant_weight(inputs.weights(d, i, wl["seed"] + 1)))
+    wq_gu, ws_gu, wq_dn, ws_dn = _FFN_ORACLE_W[key]
+    rows = max(1, min(m, threads))
+    t0 = time.perf_counter()
+    oracle.ffn_ref(np.ascontiguousarray(xb[:rows]), wq_gu, ws_gu, wq_dn, ws_dn, threads=threads)
+    t = time.perf_counter() - t0
+    flops = 2.0 * rows * d * 2 * i + 2.0 * rows * i * d
+    return flops / t / 1e12, rows, t
+
+
+def ffn_reference_arm(args):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    wl = FFN_WORKLOADS[args.workload]
+    threads = os.cpu_count() or 1
+    vals = []
+    rows = 0
+    for j in range(args.warmup + args.steps):
+        v, rows, _ = ffn_oracle_sample(wl, threads)
+        if j >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals)
+    m, d, i = wl["m"], wl["d"], wl["i"]
+    flops = 2.0 * m * d * 2 * i + 2.0 * m * i * d
+    print(json.dumps({
+        "impl": "reference", "metric": FFN_METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": flops / (value * 1e12) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "m": m, "d": d, "i": i},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{rows} of {m} token rows per step, scaled to the metric's unit"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+    return 0
+
+
+def ffn_arm(args):
+    """One step = one fp8q_ffn call: quant(x), gate|up GEMM, SiLU*up + quant, down GEMM."""
+    import torch
+    from fp8_block_scaled_group_b200 import api, inputs
+
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = FFN_WORKLOADS[args.workload]
+    m, d, i = wl["m"], wl["d"], wl["i"]
+    sets = []
+    for j in range(N_SETS):
+        xb = inputs.activations(m, d, wl["seed"] + 7919 * (rank * N_SETS + j))
+        to_dev = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
+        wgu, wsgu = api.quant_weight(to_dev(inputs.weights(2 * i, d, wl["seed"] + 2 * j)))
+        wdn, wsdn = api.quant_weight(to_dev(inputs.weights(d, i, wl["seed"] + 2 * j + 1)))
+        work = torch.empty(api.ffn_workspace_layout(m, d, i)[5], dtype=torch.uint8, device=dev)
+        sets.append(dict(x=to_dev(xb), xb=xb, w=(wgu, wsgu, wdn, wsdn), work=work,
+                         y=torch.empty((m, d), dtype=torch.bfloat16, device=dev)))
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def step(j):
+        s = sets[j % N_SETS]
+        api.ffn(s["x"], *s["w"], workspace=s["work"], out=s["y"])
+
+    counted = {}
+
+    def timed(fn, steps):
+        for j in range(args.warmup):
+            fn(j)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(int(2e6 + 2e5 * steps))
+        l0 = api.launch_count()
+        e0.record(stream)
+        for j in range(steps):
+            fn(j)
+        e1.record(stream)
+        counted[fn.__name__] = api.launch_count() - l0
+        torch.cuda.synchronize()
+        barrier(world)
+        return max_over_ranks(e0.elapsed_time(e1), world) / steps
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ms = timed(step, args.steps)
+    launches = counted["step"]
+    # The activation step alone, over each set's own gate|up output.
+    mids = [api.ffn_intermediates(s["work"], m, d, i) for s in sets]
+    act_out = [(mid["q_h"], None, mid["s_h_kmajor"]) for mid in mids]
+
+    def act(j):
+        gu = mids[j % N_SETS]["gate_up"]
+        api.silu_mul_quant(gu[:, :i], gu[:, i:], out=act_out[j % N_SETS])
+
+    act_ms = timed(act, args.steps)
+
+    def gate_up(j):
+        mid = mids[j % N_SETS]
+        s = sets[j % N_SETS]
+        api.gemm_blockscaled(mid["q_x"], mid["s_x_kmajor"], s["w"][0], s["w"][1], out=mid["gate_up"])
+
+    gu_ms = timed(gate_up, args.steps)
+    clk = clocks.stop()
+
+    x_host = [torch.from_numpy(s["xb"].view(np.int16)).view(torch.bfloat16).pin_memory() for s in sets]
+    y_host = torch.empty((m, d), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty((m, d), dtype=torch.bfloat16, device=dev)
+
+    def e2e(j):
+        s = sets[j % N_SETS]
+        x_dev.copy_(x_host[j % N_SETS], non_blocking=True)
+        api.ffn(x_dev, *s["w"], workspace=s["work"], out=s["y"])
+        y_host.copy_(s["y"], non_blocking=True)
+
+    e2e_ms = timed(e2e, args.steps)
+
+    flops = 2.0 * m * d * 2 * i + 2.0 * m * i * d
+    hbm, bf16, _, src = load_peaks()
+    fp8_peak = 2.0 * bf16
+    act_bytes = m * i * 4 + m * i + 4 * (i // 128) * (-(-m // 16) * 16)
+    gu_flops = 2.0 * m * 2 * i * d
+    if m <= 64:
+        gu_bytes = gemm_hbm_bytes(m, 2 * i, d)
+        roofline = {"bound": "hbm", "kernel": "gemm_decode_kernel (gate|up)", "achieved": gu_bytes / (gu_ms * 1e-3) / 1e9,
+                    "peak": hbm, "unit": "GB/s", "frac": gu_bytes / (gu_ms * 1e-3) / 1e9 / hbm, "traffic": None,
+                    "us": gu_ms * 1e3, "peak_source": f"{src} copy bandwidth"}
+    else:
+        tf = gu_flops / (gu_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "kernel": "gemm_blockscaled_kernel (gate|up)", "achieved": tf,
+                    "peak": fp8_peak, "unit": "TFLOP/s", "frac": tf / fp8_peak, "traffic": None,
+                    "us": gu_ms * 1e3, "peak_source": f"{src} bf16 burst x 2 (fp8:bf16 nominal ratio)"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        v, rows, t = ffn_oracle_sample(wl, threads)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{rows} of {m} token rows of one FFN step, {t:.1f} s, scaled to TFLOP/s"}
+    if rank == 0:
+        line = {
+            "metric": FFN_METRIC, "value": flops * world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "m": m, "d": d, "i": i, "parallelism": f"replicas{world}",
+                       "l2": f"{N_SETS} rotating input sets (weights {N_SETS * 3 * i * d / 1e6:.0f} MB) > L2"},
+            "roofline": roofline,
+            "act_silu_mul_quant": {"bound": "hbm", "kernel": "silu_mul_quant_kernel",
+                                   "achieved": act_bytes / (act_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                                   "frac": act_bytes / (act_ms * 1e-3) / 1e9 / hbm, "us": act_ms * 1e3,
+                                   "bytes": act_bytes},
+            "cpu_baseline": cpu,
+            "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": m * d * 2, "d2h_bytes_per_step": m * d * 2},
+            "gpu_launches": int(sum_over_ranks(launches, world)),
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    barrier(world)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(FFN_WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    if args.workload in FFN_WORKLOADS:
+        if args.impl == "reference":
+            return ffn_reference_arm(args)
+        return ffn_arm(args)
     if args.impl == "reference":
         return reference_arm(args)
     return ours_arm(args)

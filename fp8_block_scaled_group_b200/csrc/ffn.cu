@@ -13,8 +13,8 @@
 // v = p / (1 + e^-g) with the hardware exponential and reciprocal. v is
 // within a few fp32 ulps of the real value, so rounding v to bf16 gives the
 // right answer unless v lies near a bf16 rounding tie (bits 15..0 of v close
-// to 0x8000). Such values, and the ranges where the fp32 evaluation is not
-// accurate (g < -24, results outside the normal fp32 range), take the slow
+// to 0x8000). Such values, and results outside the range where the fp32
+// evaluation is accurate (|v| below 2^-126 or from 2^126 up), take the slow
 // path in fp64, which rounds exactly; for g > 32 the factor 1/(1+e^-g) is
 // within 2^-46 of 1, p is either exactly a bf16 tie or at least 2^-17 |p|
 // from one, and a tie goes toward zero because silu(g) < g.
@@ -36,7 +36,6 @@ namespace fp8q {
 
 namespace {
 
-constexpr float kFastMinGate = -24.0f;  // below: e^-g > 2^34, slow path
 
 // bf16 magnitude bits of a > 0 (finite double), nearest; ties to even, or
 // toward zero when tie_down. Overflow gives +inf (0x7F80).
@@ -91,6 +90,19 @@ __device__ __forceinline__ float rcp_approx(float x) {
     return y;
 }
 
+// Minimum and maximum that return NaN when either input is NaN.
+__device__ __forceinline__ float min_nan(float a, float b) {
+    float r;
+    asm("min.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+__device__ __forceinline__ float max_nan(float a, float b) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t bf16x2_rn(float2 v) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(v.y), "f"(v.x));
@@ -103,10 +115,11 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float2 v) {
 // part of log2(e) (Cody and Waite's argument splitting): 2^(yh + yl) =
 // 2^yh * (1 + yl ln 2) to first order in the tiny yl. The quotient is the
 // approximate reciprocal's product plus one remainder correction. The
-// result is the packed bf16 rounding of v(1 + kTieBand), which stands when
-// v(1 - kTieBand) rounds to the same value and v is in the range where the
-// evaluation is accurate; bit b of the returned *ok is set for element b.
-__device__ __forceinline__ uint32_t silu_mul_fast2(float2 g, float2 u, uint32_t* ok, float2* v_out) {
+// result is the packed bf16 rounding of v(1 + kTieBand); it stands (*ok)
+// when v(1 - kTieBand) rounds to the same pair and both |v| lie in
+// [2^-126, 2^126), where the evaluation is accurate. An overflowing g*u or
+// e^-g shows up there as an infinite, zero or NaN v.
+__device__ __forceinline__ uint32_t silu_mul_fast2(float2 g, float2 u, bool* ok, float2* v_out) {
     const float2 p = __fmul2_rn(g, u);  // exact for normal results: two 8-bit significands
     const float2 L = make_float2(kLog2eHi, kLog2eHi);
     const float2 yh = __fmul2_rn(g, L);                                   // g log2(e), rounded
@@ -120,17 +133,15 @@ __device__ __forceinline__ uint32_t silu_mul_fast2(float2 g, float2 u, uint32_t*
     const float2 v = __ffma2_rn(__ffma2_rn(make_float2(-v0.x, -v0.y), d, p), r, v0);
     const uint32_t hi = bf16x2_rn(__fmul2_rn(v, make_float2(1.0f + kTieBand, 1.0f + kTieBand)));
     const uint32_t lo = bf16x2_rn(__fmul2_rn(v, make_float2(1.0f - kTieBand, 1.0f - kTieBand)));
-    const uint32_t diff = hi ^ lo;
-    const bool ok0 = (diff & 0xFFFFu) == 0u && g.x >= kFastMinGate && fabsf(v.x) >= 0x1p-126f &&
-                     fabsf(p.x) <= 0x1.fffffep127f;
-    const bool ok1 = (diff >> 16) == 0u && g.y >= kFastMinGate && fabsf(v.y) >= 0x1p-126f &&
-                     fabsf(p.y) <= 0x1.fffffep127f;
-    *ok = (ok0 ? 1u : 0u) | (ok1 ? 2u : 0u);
+    // NaN-propagating, so a NaN v (overflowed g*u or e^-g) fails both tests
+    const float vmin = min_nan(fabsf(v.x), fabsf(v.y));
+    const float vmax = max_nan(fabsf(v.x), fabsf(v.y));
+    *ok = hi == lo && vmin >= 0x1p-126f && vmax < 0x1p126f;
     *v_out = v;
     return hi;
 }
 
-// 8 packed bf16 gates and ups -> 8 packed bf16 h. Elements the fast path
+// 8 packed bf16 gates and ups -> 8 packed bf16 h. Pairs the fast path
 // cannot settle (rare) go through the fp64 path, in a branch the whole warp
 // takes only when some lane needs it.
 __device__ __forceinline__ uint4 silu_mul8(const uint4 g, const uint4 u) {
@@ -141,17 +152,16 @@ __device__ __forceinline__ uint4 silu_mul8(const uint4 g, const uint4 u) {
     uint32_t ok = 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        uint32_t okj;
+        bool okj;
         float2 v;
         h[j] = silu_mul_fast2(make_float2(gf[2 * j], gf[2 * j + 1]), make_float2(uf[2 * j], uf[2 * j + 1]), &okj, &v);
-        ok |= okj << (2 * j);
+        ok |= (okj ? 1u : 0u) << j;
     }
-    if (__any_sync(0xFFFFFFFFu, ok != 0xFFu)) {
+    if (__any_sync(0xFFFFFFFFu, ok != 0xFu)) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            if (!(ok & (1u << (2 * j)))) h[j] = (h[j] & 0xFFFF0000u) | silu_mul_slow(gf[2 * j], uf[2 * j]);
-            if (!(ok & (2u << (2 * j)))) h[j] = (h[j] & 0x0000FFFFu) | (silu_mul_slow(gf[2 * j + 1], uf[2 * j + 1]) << 16);
-        }
+        for (int j = 0; j < 4; ++j)
+            if (!(ok & (1u << j)))
+                h[j] = silu_mul_slow(gf[2 * j], uf[2 * j]) | (silu_mul_slow(gf[2 * j + 1], uf[2 * j + 1]) << 16);
     }
     return make_uint4(h[0], h[1], h[2], h[3]);
 }
@@ -222,11 +232,11 @@ __global__ void __launch_bounds__(256) check_silu_mul_kernel(unsigned long long*
         for (uint32_t ub = threadIdx.x; ub < 0x10000u; ub += blockDim.x) {
             if ((ub & 0x7F80u) == 0x7F80u) continue;
             const float u = __uint_as_float(ub << 16);
-            uint32_t ok;
+            bool ok;
             float2 v;
             const uint32_t hf = silu_mul_fast2(make_float2(g, g), make_float2(u, u), &ok, &v) & 0xFFFFu;
             ++pairs;
-            if (!(ok & 1u)) continue;
+            if (!ok) continue;
             ++taken;
             bad += hf != silu_mul_slow(g, u);
             const double vd = static_cast<double>(g) * static_cast<double>(u) / (1.0 + exp(-static_cast<double>(g)));
