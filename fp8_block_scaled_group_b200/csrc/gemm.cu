@@ -24,7 +24,9 @@
 //               the even CTA's barrier; plus the block's 128 activation
 //               scales (one K-major row slice) into an 8-slot local ring
 //   warp 1      TMEM allocation for the pair; in the even CTA, the MMA issuer
-//   warps 2-3   idle after set-up
+//               of the even K blocks (TMEM buffer 0)
+//   warp 2      in the even CTA, the MMA issuer of the odd K blocks (buffer 1)
+//   warp 3      idle after set-up
 //   warps 4-11  promotion + epilogue. Warp w reads TMEM lanes 32*(w%4)..+31
 //               of its own CTA (its tile rows) and column half (w-4)/4 (128
 //               columns, one weight block), one row per thread
@@ -54,6 +56,7 @@ constexpr uint32_t BN = 256;       // output columns per tile
 constexpr uint32_t BN_CTA = 128;   // rows of B staged by each CTA
 constexpr uint32_t BK = 128;
 constexpr uint32_t kStages = 6;
+static_assert(kStages % 2 == 0, "each stage must always be consumed by the same MMA issuer");
 constexpr uint32_t kScaleStages = 8;
 constexpr uint32_t kThreads = 384;
 constexpr uint32_t kEpiWarps = 8;
@@ -78,11 +81,11 @@ struct __align__(1024) GemmSmem {
     uint64_t sempty[kScaleStages];
     uint64_t tfull[2];
     uint64_t tempty[2];
-    uint64_t mma_done;
+    uint64_t mma_done[2];
     uint32_t tmem_base;
     uint32_t _pad;
     uint32_t abort;
-    uint32_t consumed;  // K blocks whose TMA data the MMA thread has seen land
+    uint32_t consumed[2];  // per MMA issuer: 1 + its last K block whose TMA data it has seen land
 };
 
 constexpr size_t kSmemBytes = sizeof(GemmSmem) + 1024;  // + alignment slack
@@ -132,9 +135,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_init(&sm.tfull[b], 1);
             mbar_init(&sm.tempty[b], 2 * kEpiWarps);  // promotion warps of both CTAs
         }
-        mbar_init(&sm.mma_done, 1);
+        mbar_init(&sm.mma_done[0], 1);
+        mbar_init(&sm.mma_done[1], 1);
         sm.abort = 0;
-        sm.consumed = 0;
+        sm.consumed[0] = sm.consumed[1] = 0;
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -185,12 +189,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     issued = it + 1;
                 }
             }
-        } else if (warp == 1 && lane == 0 && rank == 0) {
+        } else if ((warp == 1 || warp == 2) && lane == 0 && rank == 0) {
+            // Two MMA issuers, one per TMEM buffer: warp 1 issues the K
+            // blocks of even index (buffer 0), warp 2 those of odd index
+            // (buffer 1). Four back-to-back tcgen05.mma hold their warp's SM
+            // sub-partition for about three MMA durations, which delays the
+            // promotion warps sharing it; alternating issuers halves that
+            // stall on each sub-partition. The two buffers' MMAs are
+            // independent, reuse of a buffer is ordered by its tempty
+            // barrier, and with an even stage count every stage is always
+            // consumed (and committed) by the same issuer.
             constexpr uint32_t idesc = idesc_e4m3_f32(BM_PAIR, BN);
+            const uint32_t par = warp - 1u;
             uint32_t it = 0;
             bool ok = true;
             for (uint32_t tile = pair; ok && tile < sh.num_tiles; tile += num_pairs) {
                 for (uint32_t kb = 0; kb < G; ++kb, ++it) {
+                    if ((it & 1u) != par) continue;
                     const uint32_t s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
                     const uint32_t b = it & 1u;
@@ -199,7 +214,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    sm.consumed = it + 1;
+                    sm.consumed[par] = it + 1;
                     if (!mbar_wait(&sm.tempty[b], tph ^ 1u, abort)) {
                         ok = false;
                         break;
@@ -216,9 +231,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
             }
             // Every MMA this thread issued has completed once mma_done fires.
-            mma_commit_pair(&sm.mma_done);
+            mma_commit_pair(&sm.mma_done[par]);
             volatile uint32_t never = 0;
-            mbar_wait(&sm.mma_done, 0, &never);
+            mbar_wait(&sm.mma_done[par], 0, &never);
         }
     } else {
         regs_inc<kRegsHigh>();
@@ -305,9 +320,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         volatile uint32_t never = 0;
         if (threadIdx.x == 0) atomicOr(&g_device_error, 1u);
         if (warp == 0 && lane == 0) {
-            if (rank == 0)
-                for (uint32_t it = sm.consumed; it < issued; ++it)
-                    mbar_wait(&sm.full[it % kStages], (it / kStages) & 1u, &never);
+            if (rank == 0) {
+                const uint32_t from = sm.consumed[0] < sm.consumed[1] ? sm.consumed[0] : sm.consumed[1];
+                for (uint32_t it = from; it < issued; ++it)
+                    if (it >= sm.consumed[it & 1u]) mbar_wait(&sm.full[it % kStages], (it / kStages) & 1u, &never);
+            }
             const uint32_t first = issued > kScaleStages ? issued - kScaleStages : 0u;
             for (uint32_t it = first; it < issued; ++it)
                 mbar_wait(&sm.sfull[it % kScaleStages], (it / kScaleStages) & 1u, &never);
