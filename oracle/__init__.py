@@ -70,6 +70,11 @@ def _load():
         lib.oracle_gemm_ref_rows.argtypes = [P, P, P, P, U32, U32, P, ctypes.c_size_t,
                                              ctypes.c_size_t, P]
         lib.oracle_gemm_ref_rows.restype = None
+        lib.oracle_gemm_ref_rows_geom.argtypes = [P, P, P, P, U32, U32, U32, U32, P, ctypes.c_size_t,
+                                                  ctypes.c_size_t, P]
+        lib.oracle_gemm_ref_rows_geom.restype = None
+        lib.oracle_quant_weight_rowwise.argtypes = [P, U32, U32, P, P]
+        lib.oracle_quant_weight_rowwise.restype = ctypes.c_int
         lib.oracle_check_tolerance.argtypes = [P, P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_double)]
         lib.oracle_check_tolerance.restype = ctypes.c_size_t
         lib.oracle_silu_mul_bf16.argtypes = [ctypes.c_uint16, ctypes.c_uint16]
@@ -143,13 +148,26 @@ def quant_weight(w_bf16: np.ndarray):
     return wq, ws
 
 
+def quant_weight_rowwise(w_bf16: np.ndarray):
+    """bf16 bits [N,K] -> (wq [N,K] u8, w_scale [N] f32), one scale per row."""
+    w = np.ascontiguousarray(w_bf16, dtype=np.uint16)
+    n, k = w.shape
+    wq = np.empty((n, k), np.uint8)
+    ws = np.empty((n,), np.float32)
+    rc = _load().oracle_quant_weight_rowwise(_ptr(w), n, k, _ptr(wq), _ptr(ws))
+    assert rc == 0
+    return wq, ws
+
+
 def gemm_ref(q: np.ndarray, a_scale_row: np.ndarray, wq: np.ndarray, w_scale: np.ndarray,
              rows: np.ndarray | None = None, threads: int = 1) -> np.ndarray:
     """Float64 reference Y[rows, N] of the block-scaled GEMM.
 
-    ``a_scale_row`` is the row-major [M, K/128] activation scale. ``rows``
-    selects output rows (default: all). ``threads`` > 1 splits the rows over
-    Python threads; the C loop itself is unchanged.
+    ``a_scale_row`` is the row-major [M, K/128] activation scale. The weight
+    scale is either block-scaled [N/128, K/128] or per row [N] (its shape
+    selects the geometry). ``rows`` selects output rows (default: all).
+    ``threads`` > 1 splits the rows over Python threads; the C loop itself
+    is unchanged.
     """
     lib = _load()
     q = np.ascontiguousarray(q, dtype=np.uint8)
@@ -158,7 +176,12 @@ def gemm_ref(q: np.ndarray, a_scale_row: np.ndarray, wq: np.ndarray, w_scale: np
     ws = np.ascontiguousarray(w_scale, dtype=np.float32)
     m, k = q.shape
     n = wq.shape[0]
-    assert wq.shape[1] == k and a_s.shape == (m, k // GROUP) and ws.shape == (n // GROUP, k // GROUP)
+    assert wq.shape[1] == k and a_s.shape == (m, k // GROUP)
+    if ws.shape == (n,):
+        block_n, block_k = 1, k
+    else:
+        assert ws.shape == (n // GROUP, k // GROUP)
+        block_n, block_k = GROUP, GROUP
     if rows is None:
         rows_arr = np.arange(m, dtype=np.int64)
     else:
@@ -166,13 +189,13 @@ def gemm_ref(q: np.ndarray, a_scale_row: np.ndarray, wq: np.ndarray, w_scale: np
         assert rows_arr.size == 0 or (rows_arr.min() >= 0 and rows_arr.max() < m)
     cnt = rows_arr.size
     ref = np.empty((cnt, n), np.float64)
-    args = (_ptr(q), _ptr(a_s), _ptr(wq), _ptr(ws), n, k, _ptr(rows_arr))
+    args = (_ptr(q), _ptr(a_s), _ptr(wq), _ptr(ws), n, k, block_n, block_k, _ptr(rows_arr))
     if threads <= 1 or cnt <= 1:
-        lib.oracle_gemm_ref_rows(*args, 0, cnt, _ptr(ref))
+        lib.oracle_gemm_ref_rows_geom(*args, 0, cnt, _ptr(ref))
     else:
         bounds = np.linspace(0, cnt, min(threads, cnt) + 1).astype(int)
         with ThreadPoolExecutor(len(bounds) - 1) as ex:
-            futs = [ex.submit(lib.oracle_gemm_ref_rows, *args, int(a), int(b - a), _ptr(ref))
+            futs = [ex.submit(lib.oracle_gemm_ref_rows_geom, *args, int(a), int(b - a), _ptr(ref))
                     for a, b in zip(bounds[:-1], bounds[1:])]
             for f in futs:
                 f.result()

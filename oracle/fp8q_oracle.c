@@ -31,6 +31,7 @@
 #include <float.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #if !defined(FLT_EVAL_METHOD) || FLT_EVAL_METHOD != 0
@@ -239,26 +240,31 @@ int oracle_quant_weight(const uint16_t *w, uint32_t n, uint32_t k,
 /*
  * Float64 dequantized reference of the block-scaled GEMM
  * (dispatch_proj.rs, `cublas_fp8_proj` / `cublas_fp8_proj_prequant`:
- * out[M,N] = act[M,K] @ weight^T, activation scales per [token, 128 of K],
- * weight scales per 128x128 block):
- *   ref[i][col] = sum_k  deq(q[r_i][k]) * a_s[r_i][k/128]
- *                      * deq(wq[col][k]) * w_s[col/128][k/128]
+ * out[M,N] = act[M,K] @ weight^T, activation scales per [token, 128 of K]),
+ * for a weight whose scales follow the block geometry of
+ * `dequant_fp8_bf16_into`: the scale of weight element [col][kk] is
+ *   w_s[(col / block_n) * (k / block_k) + kk / block_k]
+ * (block_n = block_k = 128 for the block-scaled format; block_n = 1,
+ * block_k = k for the per-row format, one multiplier per weight row):
+ *   ref[i][col] = sum_kk  deq(q[r_i][kk]) * a_s[r_i][kk/128]
+ *                       * deq(wq[col][kk]) * w_s[...]
  * for each requested row r_i (rows == NULL means rows 0..n_rows-1).
  *   q      e4m3 [m, k];  a_s  fp32 [m, k/128] row-major (the definition's
  *          own indexing; the K-major copy is a layout of the same numbers)
- *   wq     e4m3 [n, k];  w_s  fp32 [n/128, k/128]
+ *   wq     e4m3 [n, k];  w_s  fp32, indexed as above
  *   ref    float64 [n_rows, n]
  * Rows are independent; `first`/`count` select a slice of the requested
  * rows so a caller may split the work over threads.
  */
-void oracle_gemm_ref_rows(const uint8_t *q, const float *a_s,
-                          const uint8_t *wq, const float *w_s,
-                          uint32_t n, uint32_t k,
-                          const int64_t *rows, size_t first, size_t count,
-                          double *ref)
+void oracle_gemm_ref_rows_geom(const uint8_t *q, const float *a_s,
+                               const uint8_t *wq, const float *w_s,
+                               uint32_t n, uint32_t k, uint32_t block_n, uint32_t block_k,
+                               const int64_t *rows, size_t first, size_t count,
+                               double *ref)
 {
     double lut[256];
     uint32_t G = k / GROUP;
+    uint32_t sk = k / block_k;
     size_t i;
     uint32_t col, kk;
     for (i = 0; i < 256; i++)
@@ -269,13 +275,53 @@ void oracle_gemm_ref_rows(const uint8_t *q, const float *a_s,
         const float *sa = a_s + (size_t)r * G;
         for (col = 0; col < n; col++) {
             const uint8_t *qw = wq + (size_t)col * k;
-            const float *sw = w_s + (size_t)(col / GROUP) * G;
+            const float *sw = w_s + (size_t)(col / block_n) * sk;
             double acc = 0.0;
             for (kk = 0; kk < k; kk++)
-                acc += lut[qa[kk]] * (double)sa[kk / GROUP] * lut[qw[kk]] * (double)sw[kk / GROUP];
+                acc += lut[qa[kk]] * (double)sa[kk / GROUP] * lut[qw[kk]] * (double)sw[kk / block_k];
             ref[i * n + col] = acc;
         }
     }
+}
+
+/* The block-scaled case: 128 x 128 weight-scale blocks. */
+void oracle_gemm_ref_rows(const uint8_t *q, const float *a_s,
+                          const uint8_t *wq, const float *w_s,
+                          uint32_t n, uint32_t k,
+                          const int64_t *rows, size_t first, size_t count,
+                          double *ref)
+{
+    oracle_gemm_ref_rows_geom(q, a_s, wq, w_s, n, k, GROUP, GROUP, rows, first, count, ref);
+}
+
+/*
+ * Per-row FP8 weight (dispatch_proj.rs, `dequant_fp8_bf16_into`: the
+ * per-row format has block_n = 1, block_k = K, one multiplier per row).
+ * The pages take such weights from a checkpoint and do not say how they
+ * were quantized; the reading taken is the same amax / scale / code steps
+ * as every other block, over the whole row:
+ *   w        bf16 bits [n, k] row-major
+ *   wq       e4m3 codes [n, k] row-major
+ *   w_scale  fp32 [n]: max(max_j |w[r][j]|, 1e-10) / 448
+ * Returns 0, or -1 if k is 0.
+ */
+int oracle_quant_weight_rowwise(const uint16_t *w, uint32_t n, uint32_t k,
+                                uint8_t *wq, float *w_scale)
+{
+    uint32_t r, c;
+    float *row;
+    if (k == 0)
+        return -1;
+    row = (float *)malloc((size_t)k * sizeof(float));
+    if (!row)
+        return -1;
+    for (r = 0; r < n; r++) {
+        for (c = 0; c < k; c++)
+            row[c] = oracle_bf16_to_f32(w[(size_t)r * k + c]);
+        w_scale[r] = quantize_group(row, 1, k, wq + (size_t)r * k, 1);
+    }
+    free(row);
+    return 0;
 }
 
 /*
