@@ -46,6 +46,9 @@ SIGNATURES = {
     "fp8q_quant_act_variant": (ctypes.c_int, [P, P, P, P, U32, U32, I32, P]),
     "fp8q_quant_weight": (ctypes.c_int, [P, P, P, U32, U32, P]),
     "fp8q_gemm_blockscaled": (ctypes.c_int, [P, P, P, P, P, U32, U32, U32, P]),
+    "fp8q_quant_weight_rowwise": (ctypes.c_int, [P, P, P, U32, U32, P]),
+    "fp8q_gemm_ex": (ctypes.c_int, [P, P, P, P, I32, P, U32, U32, U32, P]),
+    "fp8q_linear_ex": (ctypes.c_int, [P, P, P, I32, P, P, SZ, U32, U32, U32, P]),
     "fp8q_linear_workspace_bytes": (SZ, [U32, U32]),
     "fp8q_linear_scale_offset": (SZ, [U32, U32]),
     "fp8q_linear": (ctypes.c_int, [P, P, P, P, P, SZ, U32, U32, U32, P]),

@@ -14,6 +14,7 @@ import torch
 from . import _lib
 
 AUTO, SINGLE, MULTI = 0, 1, 2
+WEIGHT_BLOCK128, WEIGHT_PER_ROW = 0, 1
 GROUP = 128
 
 
@@ -82,19 +83,40 @@ def quant_weight(w: torch.Tensor, stream=None):
     return wq, ws
 
 
+def quant_weight_rowwise(w: torch.Tensor, stream=None):
+    """w bf16 [N, K] -> (wq uint8 [N, K], w_scale fp32 [N]), one scale per weight row."""
+    n, k = w.shape
+    _need(w, torch.bfloat16, (n, k), "w")
+    wq = torch.empty((n, k), dtype=torch.uint8, device=w.device)
+    ws = torch.empty((n,), dtype=torch.float32, device=w.device)
+    _lib.check(_lib.load().fp8q_quant_weight_rowwise(_p(w), _p(wq), _p(ws), n, k, _stream(stream)),
+               "fp8q_quant_weight_rowwise")
+    return wq, ws
+
+
+def _weight_format(w_scale: torch.Tensor, n: int, k: int) -> int:
+    """The weight format its scale tensor's shape selects: [N/128, K/128] or [N]."""
+    if tuple(w_scale.shape) == (n,):
+        _need(w_scale, torch.float32, (n,), "w_scale")
+        return WEIGHT_PER_ROW
+    _need(w_scale, torch.float32, (n // GROUP, k // GROUP), "w_scale")
+    return WEIGHT_BLOCK128
+
+
 def gemm_blockscaled(q: torch.Tensor, s_kmajor: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
                      out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """q uint8 [M,K], s_kmajor fp32 [K/128, ceil16(M)], wq uint8 [N,K], w_scale fp32 [N/128,K/128] -> y bf16 [M,N]."""
+    """q uint8 [M,K], s_kmajor fp32 [K/128, ceil16(M)], wq uint8 [N,K], w_scale fp32 [N/128,K/128]
+    (block-scaled) or [N] (per row) -> y bf16 [M,N]."""
     m, k = q.shape
     n = wq.shape[0]
     _need(q, torch.uint8, (m, k), "q")
     _need(s_kmajor, torch.float32, (k // GROUP, m_pad(m)), "s_kmajor")
     _need(wq, torch.uint8, (n, k), "wq")
-    _need(w_scale, torch.float32, (n // GROUP, k // GROUP), "w_scale")
+    fmt = _weight_format(w_scale, n, k)
     y = torch.empty((m, n), dtype=torch.bfloat16, device=q.device) if out is None else out
     _need(y, torch.bfloat16, (m, n), "y")
-    _lib.check(_lib.load().fp8q_gemm_blockscaled(_p(q), _p(s_kmajor), _p(wq), _p(w_scale), _p(y), m, n, k,
-                                                  _stream(stream)), "fp8q_gemm_blockscaled")
+    _lib.check(_lib.load().fp8q_gemm_ex(_p(q), _p(s_kmajor), _p(wq), _p(w_scale), fmt, _p(y), m, n, k,
+                                         _stream(stream)), "fp8q_gemm_ex")
     return y
 
 
@@ -113,14 +135,14 @@ def linear(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor, workspace: 
     n = wq.shape[0]
     _need(x, torch.bfloat16, (m, k), "x")
     _need(wq, torch.uint8, (n, k), "wq")
-    _need(w_scale, torch.float32, (n // GROUP, k // GROUP), "w_scale")
+    fmt = _weight_format(w_scale, n, k)
     need = linear_workspace_bytes(m, k)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     y = torch.empty((m, n), dtype=torch.bfloat16, device=x.device) if out is None else out
     _need(y, torch.bfloat16, (m, n), "y")
-    _lib.check(_lib.load().fp8q_linear(_p(x), _p(wq), _p(w_scale), _p(y), _p(workspace), workspace.numel(),
-                                        m, n, k, _stream(stream)), "fp8q_linear")
+    _lib.check(_lib.load().fp8q_linear_ex(_p(x), _p(wq), _p(w_scale), fmt, _p(y), _p(workspace),
+                                           workspace.numel(), m, n, k, _stream(stream)), "fp8q_linear_ex")
     return y
 
 

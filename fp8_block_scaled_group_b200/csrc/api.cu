@@ -226,15 +226,33 @@ fp8q_status fp8q_quant_weight(const void* w, void* wq, float* w_scale, uint32_t 
     return from_cuda(launch_quant_weight(w, wq, w_scale, n, k, static_cast<cudaStream_t>(stream)));
 }
 
-fp8q_status fp8q_gemm_blockscaled(const void* q, const float* s_kmajor, const void* wq, const float* w_scale,
-                                  void* y, uint32_t m, uint32_t n, uint32_t k, void* stream) {
+fp8q_status fp8q_quant_weight_rowwise(const void* w, void* wq, float* w_scale, uint32_t n, uint32_t k,
+                                      void* stream) {
+    if (k == 0 || k % kGroup || n == 0) return FP8Q_ERR_SHAPE;
+    if (!w || !wq || !w_scale) return FP8Q_ERR_NULL;
+    if (static_cast<uint64_t>(n) * k >= (1ull << 31)) return FP8Q_ERR_SHAPE;
+    if (!aligned16(w) || !aligned16(wq) || !aligned16(w_scale)) return FP8Q_ERR_ALIGN;
+    DeviceInfo dev;
+    fp8q_status st = current_device(&dev);
+    if (st != FP8Q_OK) return st;
+    return from_cuda(launch_quant_weight_rowwise(w, wq, w_scale, n, k, static_cast<cudaStream_t>(stream)));
+}
+
+fp8q_status fp8q_gemm_ex(const void* q, const float* s_kmajor, const void* wq, const float* w_scale,
+                         int32_t weight_format, void* y, uint32_t m, uint32_t n, uint32_t k, void* stream) {
+    if (weight_format != FP8Q_WEIGHT_BLOCK128 && weight_format != FP8Q_WEIGHT_PER_ROW) return FP8Q_ERR_ARG;
     fp8q_status st = check_gemm_args(q, s_kmajor, wq, w_scale, y, m, n, k);
     if (st != FP8Q_OK) return st;
     if (m == 0) return FP8Q_OK;
     DeviceInfo dev;
     if ((st = current_device(&dev)) != FP8Q_OK) return st;
-    GemmLaunch L{q, s_kmajor, wq, w_scale, y, m, n, k, fp8q_m_pad(m), false};
+    GemmLaunch L{q, s_kmajor, wq, w_scale, y, m, n, k, fp8q_m_pad(m), false, weight_format == FP8Q_WEIGHT_PER_ROW};
     return from_cuda(launch_gemm(L, static_cast<cudaStream_t>(stream)));
+}
+
+fp8q_status fp8q_gemm_blockscaled(const void* q, const float* s_kmajor, const void* wq, const float* w_scale,
+                                  void* y, uint32_t m, uint32_t n, uint32_t k, void* stream) {
+    return fp8q_gemm_ex(q, s_kmajor, wq, w_scale, FP8Q_WEIGHT_BLOCK128, y, m, n, k, stream);
 }
 
 size_t fp8q_linear_scale_offset(uint32_t m, uint32_t k) {
@@ -246,8 +264,10 @@ size_t fp8q_linear_workspace_bytes(uint32_t m, uint32_t k) {
     return fp8q_linear_scale_offset(m, k) + round_up(g * fp8q_m_pad(m) * sizeof(float), 256);
 }
 
-fp8q_status fp8q_linear(const void* x, const void* wq, const float* w_scale, void* y, void* workspace,
-                        size_t workspace_bytes, uint32_t m, uint32_t n, uint32_t k, void* stream) {
+fp8q_status fp8q_linear_ex(const void* x, const void* wq, const float* w_scale, int32_t weight_format, void* y,
+                           void* workspace, size_t workspace_bytes, uint32_t m, uint32_t n, uint32_t k,
+                           void* stream) {
+    if (weight_format != FP8Q_WEIGHT_BLOCK128 && weight_format != FP8Q_WEIGHT_PER_ROW) return FP8Q_ERR_ARG;
     if (k == 0 || k % kGroup || n == 0 || n % kGroup) return FP8Q_ERR_SHAPE;
     if (m == 0) return FP8Q_OK;
     if (!x || !wq || !w_scale || !y || !workspace) return FP8Q_ERR_NULL;
@@ -263,8 +283,13 @@ fp8q_status fp8q_linear(const void* x, const void* wq, const float* w_scale, voi
     // The GEMM is the quantizer's programmatic dependent: its set-up (barriers,
     // TMEM, descriptor prefetch) overlaps the quantizer, and its producer waits
     // for the quantizer's grid before the first load.
-    GemmLaunch L{ws, s_k, wq, w_scale, y, m, n, k, fp8q_m_pad(m), true};
+    GemmLaunch L{ws, s_k, wq, w_scale, y, m, n, k, fp8q_m_pad(m), true, weight_format == FP8Q_WEIGHT_PER_ROW};
     return from_cuda(launch_gemm(L, static_cast<cudaStream_t>(stream)));
+}
+
+fp8q_status fp8q_linear(const void* x, const void* wq, const float* w_scale, void* y, void* workspace,
+                        size_t workspace_bytes, uint32_t m, uint32_t n, uint32_t k, void* stream) {
+    return fp8q_linear_ex(x, wq, w_scale, FP8Q_WEIGHT_BLOCK128, y, workspace, workspace_bytes, m, n, k, stream);
 }
 
 fp8q_status fp8q_silu_mul_quant(const void* gate, const void* up, uint32_t ld, void* q, float* s_row,
@@ -333,11 +358,11 @@ fp8q_status fp8q_ffn(const void* x, const void* w_gate_up, const float* w_gate_u
     // [2i, d] weight. Each later launch is the programmatic dependent of the
     // one before it and waits on it before reading its output.
     if ((st = fp8q_quant_act(x, q_x, nullptr, s_x, m, d, stream)) != FP8Q_OK) return st;
-    GemmLaunch gate_up{q_x, s_x, w_gate_up, w_gate_up_scale, gu, m, 2 * i, d, mp, true};
+    GemmLaunch gate_up{q_x, s_x, w_gate_up, w_gate_up_scale, gu, m, 2 * i, d, mp, true, false};
     if ((st = from_cuda(launch_gemm(gate_up, s))) != FP8Q_OK) return st;
     SiluLaunch act{gu, gu + i, 2 * i, q_h, nullptr, s_h, m, i, mp};
     if ((st = from_cuda(launch_silu_mul_quant(act, true, s))) != FP8Q_OK) return st;
-    GemmLaunch down{q_h, s_h, w_down, w_down_scale, y, m, d, i, mp, true};
+    GemmLaunch down{q_h, s_h, w_down, w_down_scale, y, m, d, i, mp, true, false};
     return from_cuda(launch_gemm(down, s));
 }
 

@@ -93,6 +93,7 @@ constexpr size_t kSmemBytes = sizeof(GemmSmem) + 1024;  // + alignment slack
 struct Shape {
     uint32_t M, N, G, Mp;
     uint32_t num_m, num_tiles;
+    uint32_t w_per_row;  // weight scales: 0 = [N/128, K/128] blocks, 1 = one per weight row [N]
 };
 
 __device__ __forceinline__ void tile_coords(const Shape& sh, uint32_t tile, uint32_t& m0, uint32_t& n0) {
@@ -252,20 +253,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const bool row_ok = row < sh.M;
             const uint32_t col0 = n0 + half * 128u;
             const bool col_ok = col0 < sh.N;
-            // One weight block row per warp: its G scales are one short
-            // contiguous run that stays in L1 after the first K block.
-            const float* ws_row = w_s + static_cast<size_t>(col_ok ? col0 / 128u : 0u) * G;
+            // Block-scaled weights: one weight block row per warp, whose G
+            // scales are one short contiguous run that stays in L1 after the
+            // first K block. Per-row weights: the promotion folds in the
+            // activation scale only and the epilogue applies each column's
+            // weight scale.
+            const bool per_row = sh.w_per_row != 0;
+            const float* ws_row = w_s + static_cast<size_t>(col_ok && !per_row ? col0 / 128u : 0u) * G;
             float2 acc[64];
 #pragma unroll
             for (uint32_t i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
-            float w_next = __ldg(ws_row);
+            float w_next = per_row ? 1.0f : __ldg(ws_row);
             for (uint32_t kb = 0; kb < G; ++kb, ++it) {
                 const uint32_t b = it & 1u;
                 const uint32_t tph = (it >> 1) & 1u;
                 const uint32_t ss = it % kScaleStages;
                 const uint32_t sph = (it / kScaleStages) & 1u;
                 const float w_cur = w_next;
-                if (kb + 1 < G) w_next = __ldg(ws_row + kb + 1);
+                if (!per_row && kb + 1 < G) w_next = __ldg(ws_row + kb + 1);
                 const bool got = mbar_wait(&sm.sfull[ss], sph, abort) && mbar_wait(&sm.tfull[b], tph, abort);
                 if (!__all_sync(0xFFFFFFFFu, got)) {
                     ok = false;
@@ -293,6 +298,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
             }
             if (ok && row_ok && col_ok) {
+                if (per_row) {
+                    const float4* wv = reinterpret_cast<const float4*>(w_s + col0);
+#pragma unroll
+                    for (uint32_t j = 0; j < 32; ++j) {
+                        const float4 v = __ldg(wv + j);
+                        acc[2 * j] = __fmul2_rn(acc[2 * j], make_float2(v.x, v.y));
+                        acc[2 * j + 1] = __fmul2_rn(acc[2 * j + 1], make_float2(v.z, v.w));
+                    }
+                }
                 uint4* dst = reinterpret_cast<uint4*>(y + static_cast<size_t>(row) * sh.N + col0);
 #pragma unroll
                 for (uint32_t j = 0; j < 16; ++j) {
@@ -388,6 +402,7 @@ constexpr size_t decode_smem_bytes() {
 
 struct DecodeShape {
     uint32_t M, N, G, split;
+    uint32_t w_per_row;  // weight scales: 0 = [N/128, K/128] blocks, 1 = one per weight row [N]
 };
 
 template <uint32_t NT>
@@ -520,15 +535,18 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             mbar_wait(&sm.mma_done, 0, &never);
         }
     } else {
-        const float* ws_row = w_s + static_cast<size_t>(nb) * G;
+        // Per-row weights: the weight scale is applied once, after the
+        // split-K reduction.
+        const bool per_row = sh.w_per_row != 0;
+        const float* ws_row = w_s + static_cast<size_t>(per_row ? 0u : nb) * G;
         const uint32_t lane_off = ((warp & 3u) * 32u) << 16;
-        float w_next = nk > 0 ? __ldg(ws_row + kb0) : 0.0f;
+        float w_next = per_row ? 1.0f : (nk > 0 ? __ldg(ws_row + kb0) : 0.0f);
         for (uint32_t it = 0; it < nk; ++it) {
             const uint32_t s = it % kDecStages;
             const uint32_t b = it % kDecBufs;
             const uint32_t tph = (it / kDecBufs) & 1u;
             const float wsc = w_next;
-            if (it + 1 < nk) w_next = __ldg(ws_row + kb0 + it + 1);
+            if (!per_row && it + 1 < nk) w_next = __ldg(ws_row + kb0 + it + 1);
             const bool got = mbar_wait(&sm.tfull[b], tph, abort);
             if (!__all_sync(0xFFFFFFFFu, got)) break;
             tc_fence_after();
@@ -574,6 +592,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     if (threadIdx.x < BM && !*abort) {
         const uint32_t j = threadIdx.x;
         const uint32_t red_addr = smem_addr(red);
+        const float w_row = sh.w_per_row ? __ldg(w_s + n0 + j) : 1.0f;
         for (uint32_t t = rank; t < sh.M; t += sh.split) {
             // Issue every peer's load before adding (independent remote
             // reads in flight together), then sum in rank order.
@@ -584,6 +603,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             float sum = 0.0f;
 #pragma unroll
             for (uint32_t p = 0; p < kDecMaxSplit; ++p) sum += part[p];
+            if (sh.w_per_row) sum *= w_row;
             __nv_bfloat16 h = __float2bfloat16_rn(sum);
             y[static_cast<size_t>(t) * sh.N + n0 + j] = *reinterpret_cast<uint16_t*>(&h);
         }
@@ -720,6 +740,7 @@ cudaError_t launch_decode(const GemmLaunch& L, int sms, cudaStream_t stream) {
     sh.M = L.m;
     sh.N = L.n;
     sh.G = L.k / BK;
+    sh.w_per_row = L.w_per_row ? 1u : 0u;
     const uint32_t slices = L.n / BM;
     const uint32_t split = decode_split(slices, sh.G, sms);
     sh.split = split;
@@ -759,6 +780,7 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream) {
     sh.Mp = L.mp;
     sh.num_m = (L.m + BM_PAIR - 1) / BM_PAIR;
     sh.num_tiles = sh.num_m * ((L.n + BN - 1) / BN);
+    sh.w_per_row = L.w_per_row ? 1u : 0u;
     const uint32_t max_pairs = static_cast<uint32_t>(ks.sms) / 2;
     const uint32_t grid = 2 * (sh.num_tiles < max_pairs ? sh.num_tiles : max_pairs);
     cudaLaunchConfig_t cfg = {};

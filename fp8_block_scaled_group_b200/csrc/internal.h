@@ -32,6 +32,8 @@ struct QuantLaunch {
 cudaError_t launch_quant_act(const QuantLaunch& L, cudaStream_t stream);
 cudaError_t launch_quant_weight(const void* w, void* wq, float* w_scale, uint32_t n, uint32_t k,
                                 cudaStream_t stream);
+cudaError_t launch_quant_weight_rowwise(const void* w, void* wq, float* w_scale, uint32_t n, uint32_t k,
+                                        cudaStream_t stream);
 cudaError_t launch_convert_e4m3(const float* in, uint8_t* out, size_t n, cudaStream_t stream);
 cudaError_t launch_check_division(unsigned long long* counts, cudaStream_t stream);
 
@@ -42,7 +44,8 @@ struct GemmLaunch {
     const float* w_scale;
     void* y;
     uint32_t m, n, k, mp;
-    bool pdl;  // launched as the programmatic dependent of the kernel before it
+    bool pdl;        // launched as the programmatic dependent of the kernel before it
+    bool w_per_row;  // w_scale holds one scale per weight row [n] instead of [n/128, k/128] blocks
 };
 
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream);

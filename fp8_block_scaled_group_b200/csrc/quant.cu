@@ -146,6 +146,32 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const uint16_t* __res
     if (threadIdx.x == 0) w_scale[static_cast<size_t>(bn) * G + bg] = s;
 }
 
+// Per-row weights (scale block 1 x K): one CTA of 256 threads per row. The
+// row's amax is reduced over the whole row, then the row is read again and
+// encoded with that one scale.
+__global__ void __launch_bounds__(256) quant_weight_rowwise_kernel(const uint16_t* __restrict__ w,
+                                                                   uint8_t* __restrict__ wq,
+                                                                   float* __restrict__ w_scale, uint32_t k) {
+    __shared__ float red[8];
+    const size_t base = static_cast<size_t>(blockIdx.x) * k;
+    float amax = 0.0f;
+    for (uint32_t c = threadIdx.x * 8u; c < k; c += 256u * 8u) amax = fmaxf(amax, absmax8_bits(ld_stream16(w + base + c)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = red[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+    const float s = group_scale(amax);
+    for (uint32_t c = threadIdx.x * 8u; c < k; c += 256u * 8u) {
+        float f[8];
+        widen8(*reinterpret_cast<const uint4*>(w + base + c), f);
+        *reinterpret_cast<uint2*>(wq + base + c) = encode8(f, s);
+    }
+    if (threadIdx.x == 0) w_scale[blockIdx.x] = s;
+}
+
 // Element-wise fp32 -> e4m3 with the conversion the quantizers use.
 __global__ void convert_e4m3_kernel(const float* __restrict__ in, uint8_t* __restrict__ out, size_t n) {
     const size_t pairs = (n + 1) / 2;
@@ -217,6 +243,14 @@ cudaError_t launch_quant_weight(const void* w, void* wq, float* w_scale, uint32_
     dim3 grid(k / 128, n / 128);
     quant_weight_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(w), static_cast<uint8_t*>(wq),
                                                   w_scale, k);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_weight_rowwise(const void* w, void* wq, float* w_scale, uint32_t n, uint32_t k,
+                                        cudaStream_t stream) {
+    quant_weight_rowwise_kernel<<<n, 256, 0, stream>>>(static_cast<const uint16_t*>(w), static_cast<uint8_t*>(wq),
+                                                       w_scale, k);
     note_launch();
     return cudaGetLastError();
 }

@@ -168,6 +168,41 @@ fp8q_status fp8q_gemm_blockscaled(const void *q, const float *s_kmajor, const vo
                                   uint32_t m, uint32_t n, uint32_t k, void *stream);
 
 /*
+ * Weight formats: the geometry of the weight scales (P-DP,
+ * `dequant_fp8_bf16_into`: one rule, scale[(n/block_n)*(K/block_k) + k/block_k],
+ * serves both layouts):
+ *   FP8Q_WEIGHT_BLOCK128  block_n = block_k = 128: w_scale fp32 [n/128, k/128]
+ *   FP8Q_WEIGHT_PER_ROW   block_n = 1, block_k = K: w_scale fp32 [n], one
+ *                         multiplier per weight row (the compressed-tensors
+ *                         per-row checkpoint format the pages name)
+ */
+enum { FP8Q_WEIGHT_BLOCK128 = 0, FP8Q_WEIGHT_PER_ROW = 1 };
+
+/*
+ * Per-row weight quantization: for each row r of w bf16 [n, k],
+ *   w_scale[r] = max(max_j |w[r][j]|, 1e-10f) / 448.0f,
+ *   wq[r][j]   = e4m3_rne_satfinite(w[r][j] / w_scale[r]),
+ * the activation quantizer's arithmetic over a 1 x k block. (The pages load
+ * such weights from a checkpoint; the quantizer is this library's.)
+ * k a multiple of 128; n*k below 2^31.
+ * Errors: NULL, ALIGN, SHAPE, UNSUPPORTED_DEVICE, CUDA.
+ */
+fp8q_status fp8q_quant_weight_rowwise(const void *w, void *wq, float *w_scale,
+                                      uint32_t n, uint32_t k, void *stream);
+
+/*
+ * fp8q_gemm_blockscaled for either weight format:
+ *   y[t][c] = bf16_rn( sum_g s_kmajor[g][t] * ws(c, g)
+ *                      * sum_{j<128} q[t][128g+j] * wq[c][128g+j] )
+ * with ws(c, g) = w_scale[c/128][g] (FP8Q_WEIGHT_BLOCK128) or w_scale[c]
+ * (FP8Q_WEIGHT_PER_ROW; applied once per output after the sum over g).
+ * Errors: as fp8q_gemm_blockscaled, plus ARG for an unknown format.
+ */
+fp8q_status fp8q_gemm_ex(const void *q, const float *s_kmajor, const void *wq,
+                         const float *w_scale, int32_t weight_format, void *y,
+                         uint32_t m, uint32_t n, uint32_t k, void *stream);
+
+/*
  * Workspace bytes fp8q_linear needs for (m, k): the FP8 activation
  * [m, k] at offset 0, then the K-major scales [k/128, ceil16(m)] fp32 at
  * offset fp8q_linear_scale_offset(m, k).
@@ -188,6 +223,12 @@ size_t fp8q_linear_scale_offset(uint32_t m, uint32_t k);
 fp8q_status fp8q_linear(const void *x, const void *wq, const float *w_scale, void *y,
                         void *workspace, size_t workspace_bytes,
                         uint32_t m, uint32_t n, uint32_t k, void *stream);
+
+/* fp8q_linear for either weight format (see fp8q_gemm_ex). */
+fp8q_status fp8q_linear_ex(const void *x, const void *wq, const float *w_scale,
+                           int32_t weight_format, void *y,
+                           void *workspace, size_t workspace_bytes,
+                           uint32_t m, uint32_t n, uint32_t k, void *stream);
 
 /*
  * fp8q_linear for callers that cannot allocate device memory. The paper has
