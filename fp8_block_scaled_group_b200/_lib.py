@@ -49,6 +49,7 @@ SIGNATURES = {
     "fp8q_quant_weight_rowwise": (ctypes.c_int, [P, P, P, U32, U32, P]),
     "fp8q_gemm_ex": (ctypes.c_int, [P, P, P, P, I32, P, U32, U32, U32, P]),
     "fp8q_linear_ex": (ctypes.c_int, [P, P, P, I32, P, P, SZ, U32, U32, U32, P]),
+    "fp8q_linear_decode_fused": (ctypes.c_int, [P, P, P, I32, P, P, SZ, U32, U32, U32, P]),
     "fp8q_linear_workspace_bytes": (SZ, [U32, U32]),
     "fp8q_linear_scale_offset": (SZ, [U32, U32]),
     "fp8q_linear": (ctypes.c_int, [P, P, P, P, P, SZ, U32, U32, U32, P]),

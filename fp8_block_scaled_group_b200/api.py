@@ -229,6 +229,27 @@ def check_silu_mul(stream=None) -> tuple[int, int, int, float]:
     return int(a), int(b), int(c), worst
 
 
+def linear_decode_fused(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
+                        workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """linear() at decode widths (M <= 32) in one launch: the decode GEMM quantizes x itself.
+    Bit-identical to linear(); slower on B200 (see fp8q_linear_decode_fused)."""
+    m, k = x.shape
+    n = wq.shape[0]
+    _need(x, torch.bfloat16, (m, k), "x")
+    _need(wq, torch.uint8, (n, k), "wq")
+    fmt = _weight_format(w_scale, n, k)
+    need = linear_workspace_bytes(m, k)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _need(y, torch.bfloat16, (m, n), "y")
+    _lib.check(_lib.load().fp8q_linear_decode_fused(_p(x), _p(wq), _p(w_scale), fmt, _p(y), _p(workspace),
+                                                     workspace.numel(), m, n, k, _stream(stream)),
+               "fp8q_linear_decode_fused")
+    return y
+
+
 def convert_e4m3(t: torch.Tensor, stream=None) -> torch.Tensor:
     """fp32 CUDA tensor -> uint8 e4m3 codes with the quantizers' conversion."""
     if not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():

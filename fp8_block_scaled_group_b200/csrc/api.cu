@@ -279,11 +279,32 @@ fp8q_status fp8q_linear_ex(const void* x, const void* wq, const float* w_scale, 
     if (st != FP8Q_OK) return st;
     if ((st = check_gemm_args(ws, s_k, wq, w_scale, y, m, n, k)) != FP8Q_OK) return st;
     if (m == 0) return FP8Q_OK;
+    const bool per_row = weight_format == FP8Q_WEIGHT_PER_ROW;
     if ((st = fp8q_quant_act(x, ws, nullptr, s_k, m, k, stream)) != FP8Q_OK) return st;
     // The GEMM is the quantizer's programmatic dependent: its set-up (barriers,
     // TMEM, descriptor prefetch) overlaps the quantizer, and its producer waits
     // for the quantizer's grid before the first load.
-    GemmLaunch L{ws, s_k, wq, w_scale, y, m, n, k, fp8q_m_pad(m), true, weight_format == FP8Q_WEIGHT_PER_ROW};
+    GemmLaunch L{ws, s_k, wq, w_scale, y, m, n, k, fp8q_m_pad(m), true, per_row};
+    return from_cuda(launch_gemm(L, static_cast<cudaStream_t>(stream)));
+}
+
+fp8q_status fp8q_linear_decode_fused(const void* x, const void* wq, const float* w_scale, int32_t weight_format,
+                                     void* y, void* workspace, size_t workspace_bytes, uint32_t m, uint32_t n,
+                                     uint32_t k, void* stream) {
+    if (weight_format != FP8Q_WEIGHT_BLOCK128 && weight_format != FP8Q_WEIGHT_PER_ROW) return FP8Q_ERR_ARG;
+    if (k == 0 || k % kGroup || n == 0 || n % kGroup || m > kFusedDecodeMaxTokens) return FP8Q_ERR_SHAPE;
+    if (m == 0) return FP8Q_OK;
+    if (!x || !wq || !w_scale || !y || !workspace) return FP8Q_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FP8Q_ERR_WORKSPACE;
+    if (workspace_bytes < fp8q_linear_workspace_bytes(m, k)) return FP8Q_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* s_k = reinterpret_cast<float*>(ws + fp8q_linear_scale_offset(m, k));
+    fp8q_status st = check_quant_args(x, ws, nullptr, s_k, m, k);
+    if (st != FP8Q_OK) return st;
+    if ((st = check_gemm_args(ws, s_k, wq, w_scale, y, m, n, k)) != FP8Q_OK) return st;
+    DeviceInfo dev;
+    if ((st = current_device(&dev)) != FP8Q_OK) return st;
+    GemmLaunch L{ws, s_k, wq, w_scale, y, m, n, k, fp8q_m_pad(m), false, weight_format == FP8Q_WEIGHT_PER_ROW, x};
     return from_cuda(launch_gemm(L, static_cast<cudaStream_t>(stream)));
 }
 

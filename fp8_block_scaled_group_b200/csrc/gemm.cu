@@ -39,6 +39,7 @@
 #include <cstdlib>
 #include <mutex>
 
+#include "group_quant.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -372,6 +373,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // TMEM allocator and MMA issuer, warps 2-5 promotion (warp w reads TMEM
 // lanes 32*(w%4)..+31). A stage is freed after five arrivals: the MMA's
 // commit and the four promotion warps that read its token scales.
+//
+// FUSE (M <= 32): the activation quantizer runs inside this kernel. Four
+// more warps (6-9) read each K block of the bf16 activation X [M, K] (from
+// L2) and write its FP8 codes straight into the stage's token tile, in the
+// 128-byte-swizzled K-major layout the MMA descriptor expects, and its
+// per-token scales into the stage's scale slot, with the quantizer's own
+// group arithmetic (the bytes equal fp8q_quant_act's). Every weight slice
+// quantizes the same X blocks; the CTAs of slice 0 also store the codes and
+// K-major scales (pad rows zeroed) to global memory, so the call leaves the
+// same workspace as the unfused path. A stage then fills on five arrivals:
+// the weight copy's expect-tx and the four quantizer warps, whose generic
+// shared-memory writes are fenced to the async proxy first.
 
 constexpr uint32_t kDecStages = 4;
 constexpr uint32_t kDecBufs = 4;
@@ -379,6 +392,9 @@ constexpr uint32_t kDecThreads = 192;
 constexpr uint32_t kDecEpiWarps = 4;
 constexpr uint32_t kDecMaxSplit = 8;
 constexpr uint32_t kDecMaxTokens = 64;
+constexpr uint32_t kDecQuantWarps = 4;
+constexpr uint32_t kDecFusedThreads = kDecThreads + 32 * kDecQuantWarps;
+constexpr uint32_t kDecFusedMaxTokens = 32;
 
 template <uint32_t NT>
 struct __align__(1024) DecodeSmem {
@@ -401,7 +417,7 @@ constexpr size_t decode_smem_bytes() {
 }
 
 struct DecodeShape {
-    uint32_t M, N, G, split;
+    uint32_t M, N, G, split, Mp;
     uint32_t w_per_row;  // weight scales: 0 = [N/128, K/128] blocks, 1 = one per weight row [N]
 };
 
@@ -441,11 +457,13 @@ __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
     return v;
 }
 
-template <uint32_t NT>
-__global__ void __launch_bounds__(kDecThreads, 2)
+template <uint32_t NT, bool FUSE>
+__global__ void __launch_bounds__(FUSE ? kDecFusedThreads : kDecThreads, 2)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmT,
                        const __grid_constant__ CUtensorMap tmS, const float* __restrict__ w_s,
-                       uint16_t* __restrict__ y, const DecodeShape sh) {
+                       uint16_t* __restrict__ y, const DecodeShape sh, const uint16_t* __restrict__ x,
+                       uint8_t* __restrict__ q_out, float* __restrict__ s_out) {
+    static_assert(!FUSE || NT <= kDecFusedMaxTokens, "the fused quantizer serves at most 32 tokens");
     extern __shared__ uint8_t smem_raw[];
     using Smem = DecodeSmem<NT>;
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -462,7 +480,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 
     if (threadIdx.x == 0) {
         for (uint32_t s = 0; s < kDecStages; ++s) {
-            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.full[s], FUSE ? 1 + kDecQuantWarps : 1);
             mbar_init(&sm.empty[s], 1 + kDecEpiWarps);
         }
         for (uint32_t b = 0; b < kDecBufs; ++b) {
@@ -502,10 +520,15 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                 const uint32_t s = it % kDecStages;
                 const uint32_t ph = (it / kDecStages) & 1u;
                 if (!mbar_wait(&sm.empty[s], ph ^ 1u, abort)) break;
-                mbar_arrive_expect_tx(&sm.full[s], BM * BK + NT * BK + NT * 4);
-                tma_load_2d(sm.w[s], &tmW, &sm.full[s], static_cast<int32_t>(kb * BK), static_cast<int32_t>(n0));
-                tma_load_2d(sm.t[s], &tmT, &sm.full[s], static_cast<int32_t>(kb * BK), 0);
-                tma_load_2d(sm.t_scale[s], &tmS, &sm.full[s], 0, static_cast<int32_t>(kb));
+                if (FUSE) {
+                    mbar_arrive_expect_tx(&sm.full[s], BM * BK);
+                    tma_load_2d(sm.w[s], &tmW, &sm.full[s], static_cast<int32_t>(kb * BK), static_cast<int32_t>(n0));
+                } else {
+                    mbar_arrive_expect_tx(&sm.full[s], BM * BK + NT * BK + NT * 4);
+                    tma_load_2d(sm.w[s], &tmW, &sm.full[s], static_cast<int32_t>(kb * BK), static_cast<int32_t>(n0));
+                    tma_load_2d(sm.t[s], &tmT, &sm.full[s], static_cast<int32_t>(kb * BK), 0);
+                    tma_load_2d(sm.t_scale[s], &tmS, &sm.full[s], 0, static_cast<int32_t>(kb));
+                }
                 issued = it + 1;
             }
         }
@@ -534,7 +557,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             volatile uint32_t never = 0;
             mbar_wait(&sm.mma_done, 0, &never);
         }
-    } else {
+    } else if (warp < 2 + kDecEpiWarps) {
         // Per-row weights: the weight scale is applied once, after the
         // split-K reduction.
         const bool per_row = sh.w_per_row != 0;
@@ -561,6 +584,70 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                 mbar_arrive(&sm.empty[s]);  // this warp is done with the stage's token scales
             }
         }
+    } else if (FUSE) {
+        // Quantizer warps: sixteen threads own one token's 128-element group
+        // (16 bytes of X each), eight tokens at a time.
+        const uint32_t qt = threadIdx.x - kDecThreads;  // 0..127
+        const uint32_t gi = qt >> 4;
+        const uint32_t l = qt & 15u;
+        const uint32_t half_mask = 0xFFFFu << (16u * (gi & 1u));
+        const uint32_t K = G * BK;
+        // Token rows past M stay zero (codes and scales) in every stage.
+        for (uint32_t idx = qt; idx < kDecStages * (NT - sh.M) * 8u; idx += 32u * kDecQuantWarps) {
+            const uint32_t st = idx / ((NT - sh.M) * 8u);
+            const uint32_t r = idx % ((NT - sh.M) * 8u);
+            *reinterpret_cast<uint4*>(&sm.t[st][(sh.M + r / 8u) * BK + (r % 8u) * 16u]) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        for (uint32_t idx = qt; idx < kDecStages * NT; idx += 32u * kDecQuantWarps)
+            if (idx % NT >= sh.M) sm.t_scale[idx / NT][idx % NT] = 0.0f;
+        // Token t = gi + 8 r of round r. The X loads of the next K block are
+        // issued before waiting for this one's stage, so their L2 latency
+        // overlaps the wait and this block's arithmetic.
+        constexpr uint32_t R = NT / 8u;
+        uint4 cur[R], nxt[R];
+        auto load_block = [&](uint32_t kb, uint4 (&v)[R]) {
+#pragma unroll
+            for (uint32_t r = 0; r < R; ++r) {
+                const uint32_t t = gi + 8u * r;
+                v[r] = t < sh.M ? ld_stream16(x + static_cast<size_t>(t) * K + static_cast<size_t>(kb) * BK + l * 8u)
+                                : make_uint4(0u, 0u, 0u, 0u);
+            }
+        };
+        if (nk > 0) load_block(kb0, cur);
+        for (uint32_t it = 0; it < nk; ++it) {
+            const uint32_t kb = kb0 + it;
+            const uint32_t s = it % kDecStages;
+            const uint32_t ph = (it / kDecStages) & 1u;
+            if (it + 1 < nk) load_block(kb + 1, nxt);
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.empty[s], ph ^ 1u, abort))) break;
+#pragma unroll
+            for (uint32_t r = 0; r < R; ++r) {
+                const uint32_t t = gi + 8u * r;
+                if (t >= sh.M) continue;  // the same for the sixteen threads of a token
+                const size_t src = static_cast<size_t>(t) * K + static_cast<size_t>(kb) * BK + l * 8u;
+                float amax = absmax8_bits(cur[r]);
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(half_mask, amax, o));
+                const float scale = group_scale(amax);
+                float f[8];
+                widen8(cur[r], f);
+                const uint2 c = encode8(f, scale);
+                // 128-byte swizzle: 16-byte chunk j of row t sits at chunk j ^ (t % 8)
+                *reinterpret_cast<uint2*>(&sm.t[s][t * BK + ((((l >> 1) ^ (t & 7u)) << 4) | ((l & 1u) << 3))]) = c;
+                if (l == 0) sm.t_scale[s][t] = scale;
+                if (nb == 0) {
+                    st_stream8(q_out + src, c);
+                    if (l == 0) s_out[static_cast<size_t>(kb) * sh.Mp + t] = scale;
+                }
+            }
+            if (nb == 0 && qt < sh.Mp - sh.M) s_out[static_cast<size_t>(kb) * sh.Mp + sh.M + qt] = 0.0f;
+            // make the generic-proxy shared-memory writes visible to the MMA
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if ((threadIdx.x & 31u) == 0) mbar_arrive(&sm.full[s]);
+#pragma unroll
+            for (uint32_t r = 0; r < R; ++r) cur[r] = nxt[r];
+        }
     }
 
     // After a timed-out wait, let the copies this CTA started land (bounded).
@@ -584,7 +671,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     // this CTA's partial, transposed: red[t][row] (consecutive threads write
     // consecutive words).
     float* red = reinterpret_cast<float*>(&sm.w[0][0]);
-    if (warp >= 2) {
+    if (warp >= 2 && warp < 2 + kDecEpiWarps) {
 #pragma unroll
         for (uint32_t i = 0; i < NT; ++i) red[i * BM + r_local] = acc[i];
     }
@@ -700,12 +787,12 @@ cudaError_t read_clear_device_error(uint32_t* code, cudaStream_t stream) {
     return e;
 }
 
-template <uint32_t NT>
+template <uint32_t NT, bool FUSE>
 cudaError_t decode_smem_optin() {
     static std::once_flag once;
     static cudaError_t err = cudaSuccess;
     std::call_once(once, [] {
-        err = cudaFuncSetAttribute(gemm_decode_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        err = cudaFuncSetAttribute(gemm_decode_kernel<NT, FUSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    static_cast<int>(decode_smem_bytes<NT>()));
     });
     return err;
@@ -728,9 +815,9 @@ uint32_t decode_split(uint32_t slices, uint32_t G, int sms) {
     return s < limit ? s : limit;
 }
 
-template <uint32_t NT>
+template <uint32_t NT, bool FUSE>
 cudaError_t launch_decode(const GemmLaunch& L, int sms, cudaStream_t stream) {
-    const cudaError_t attr_err = decode_smem_optin<NT>();
+    const cudaError_t attr_err = decode_smem_optin<NT, FUSE>();
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap tw, tt, ts;
     if (!make_map_u8(&tw, L.wq, L.k, L.n, BM) || !make_map_u8(&tt, L.q, L.k, L.m, NT) ||
@@ -740,13 +827,14 @@ cudaError_t launch_decode(const GemmLaunch& L, int sms, cudaStream_t stream) {
     sh.M = L.m;
     sh.N = L.n;
     sh.G = L.k / BK;
+    sh.Mp = L.mp;
     sh.w_per_row = L.w_per_row ? 1u : 0u;
     const uint32_t slices = L.n / BM;
     const uint32_t split = decode_split(slices, sh.G, sms);
     sh.split = split;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(split, slices, 1);
-    cfg.blockDim = dim3(kDecThreads, 1, 1);
+    cfg.blockDim = dim3(FUSE ? kDecFusedThreads : kDecThreads, 1, 1);
     cfg.dynamicSmemBytes = decode_smem_bytes<NT>();
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
@@ -758,8 +846,9 @@ cudaError_t launch_decode(const GemmLaunch& L, int sms, cudaStream_t stream) {
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = L.pdl ? 2 : 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_decode_kernel<NT>, tw, tt, ts, L.w_scale,
-                                       static_cast<uint16_t*>(L.y), sh);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_decode_kernel<NT, FUSE>, tw, tt, ts, L.w_scale,
+                                       static_cast<uint16_t*>(L.y), sh, static_cast<const uint16_t*>(L.x),
+                                       static_cast<uint8_t*>(const_cast<void*>(L.q)), const_cast<float*>(L.s_k));
     note_launch();
     return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -767,8 +856,13 @@ cudaError_t launch_decode(const GemmLaunch& L, int sms, cudaStream_t stream) {
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream) {
     const KernelSetup& ks = setup_for_device();
     if (ks.err != cudaSuccess) return ks.err;
-    if (L.m <= 32) return launch_decode<32>(L, ks.sms, stream);
-    if (L.m <= kDecMaxTokens) return launch_decode<64>(L, ks.sms, stream);
+    if (L.x) {
+        // the quantizer runs inside the decode kernel (q and s_k are outputs)
+        if (L.m > kDecFusedMaxTokens) return cudaErrorInvalidValue;
+        return launch_decode<32, true>(L, ks.sms, stream);
+    }
+    if (L.m <= 32) return launch_decode<32, false>(L, ks.sms, stream);
+    if (L.m <= kDecMaxTokens) return launch_decode<64, false>(L, ks.sms, stream);
     CUtensorMap ta, tb, ts;
     if (!make_map_u8(&ta, L.q, L.k, L.m, BM) || !make_map_u8(&tb, L.wq, L.k, L.n, BN_CTA) ||
         !make_map_scales_box(&ts, L.s_k, L.mp, L.k / BK, BM))

@@ -46,9 +46,13 @@ struct GemmLaunch {
     uint32_t m, n, k, mp;
     bool pdl;        // launched as the programmatic dependent of the kernel before it
     bool w_per_row;  // w_scale holds one scale per weight row [n] instead of [n/128, k/128] blocks
+    // Non-null (m <= 32 only): the bf16 activation [m, k]; the decode kernel
+    // quantizes it itself and writes q and the K-major s_k as outputs.
+    const void* x = nullptr;
 };
 
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream);
+constexpr uint32_t kFusedDecodeMaxTokens = 32;
 
 // SiLU(gate) * up rounded to bf16, then quantized per 128-group of tokens.
 struct SiluLaunch {

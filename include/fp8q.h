@@ -224,6 +224,22 @@ fp8q_status fp8q_linear(const void *x, const void *wq, const float *w_scale, voi
                         void *workspace, size_t workspace_bytes,
                         uint32_t m, uint32_t n, uint32_t k, void *stream);
 
+/*
+ * fp8q_linear_ex at decode widths (m <= 32) in ONE launch: the decode GEMM
+ * quantizes x itself, K block by K block, straight into its shared-memory
+ * operand tiles (page P-DP's decode path quantizes in a separate launch).
+ * Results are bit-identical to fp8q_linear_ex, including the FP8 bytes and
+ * K-major scales it leaves in the workspace. Every weight slice of the GEMM
+ * quantizes the same activation blocks, so this path does more arithmetic:
+ * on B200 it measured slower than the two-launch fp8q_linear_ex (21.0 vs
+ * 12.4 us at m=25, n=6144, k=5120), which therefore remains the default.
+ * Errors: as fp8q_linear_ex; SHAPE also when m > 32.
+ */
+fp8q_status fp8q_linear_decode_fused(const void *x, const void *wq, const float *w_scale,
+                                     int32_t weight_format, void *y,
+                                     void *workspace, size_t workspace_bytes,
+                                     uint32_t m, uint32_t n, uint32_t k, void *stream);
+
 /* fp8q_linear for either weight format (see fp8q_gemm_ex). */
 fp8q_status fp8q_linear_ex(const void *x, const void *wq, const float *w_scale,
                            int32_t weight_format, void *y,

@@ -266,7 +266,8 @@ def test_gemm_wrong_scale_layout_fails():
 
 # ------------------------------------------------------------- linear --
 
-@pytest.mark.parametrize("m,n,k", [(16, 512, 512), (25, 6144, 5120), (1, 256, 17408), (300, 384, 1024)])
+@pytest.mark.parametrize("m,n,k", [(16, 512, 512), (25, 6144, 5120), (1, 256, 17408), (17, 5120, 17408),
+                                   (32, 256, 640), (31, 128, 1152), (33, 256, 640), (300, 384, 1024)])
 def test_linear_matches_quant_then_gemm(m, n, k):
     xb, q, s_row, s_k = oracle_act(m, k, 77, 0.01, 20.0)
     wb, wq_o, ws_o = oracle_w(n, k, 77)
@@ -290,6 +291,38 @@ def test_linear_matches_quant_then_gemm(m, n, k):
     ref = oracle.gemm_ref(q, s_row, wq_o, ws_o, rows=rows, threads=8)
     bad, worst = oracle.check_tolerance(bf16_bits(y)[rows], ref)
     assert bad == 0, worst
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 256, 17408), (16, 512, 512), (17, 5120, 17408), (25, 6144, 5120),
+                                   (31, 128, 1152), (32, 256, 640)])
+@pytest.mark.parametrize("per_row", [False, True], ids=["block128", "per_row"])
+def test_linear_decode_fused_is_linear(m, n, k, per_row):
+    """The one-launch decode path: same y bits, same workspace bytes."""
+    xb, q, s_row, s_k = oracle_act(m, k, 91, 0.01, 20.0)
+    wb = inputs.weights(n, k, 91)
+    wq_o, ws_o = oracle.quant_weight_rowwise(wb) if per_row else oracle.quant_weight(wb)
+    x = to_dev_bf16(xb)
+    wq_d = torch.from_numpy(wq_o).to(DEV)
+    ws_d = torch.from_numpy(ws_o).to(DEV)
+    need = api.linear_workspace_bytes(m, k)
+    ws_raw, workspace = guarded(need, torch.uint8, (need,))
+    y = api.linear_decode_fused(x, wq_d, ws_d, workspace=workspace)
+    y2 = api.linear(x, wq_d, ws_d)
+    torch.cuda.synchronize()
+    assert guard_intact(ws_raw, need)
+    w = workspace.cpu().numpy()
+    off = api.linear_scale_offset(m, k)
+    g, mp = k // 128, api.m_pad(m)
+    assert np.array_equal(w[:m * k].reshape(m, k), q)
+    assert np.array_equal(w[off:off + 4 * g * mp].view(np.uint32).reshape(g, mp), s_k.view(np.uint32))
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+
+
+def test_linear_decode_fused_rejects_wide_m():
+    a = torch.zeros(1 << 20, dtype=torch.uint8, device=DEV)
+    st = api._lib.load().fp8q_linear_decode_fused(api._p(a), api._p(a), api._p(a), 0, api._p(a), api._p(a),
+                                                  a.numel(), 33, 128, 128, None)
+    assert st == 2
 
 
 def test_no_device_error_flag():
