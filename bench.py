@@ -74,19 +74,33 @@ def gemm_hbm_bytes(m, n, k):
     return m * k + n * k + 4 * g * mp + 4 * (n // 128) * g + 2 * m * n
 
 
-def read_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch recorded from an ncu capture in profiles/traffic.txt,
-    or None when absent or when the kernel sources changed since the capture."""
-    path = os.path.join(ROOT, "profiles", "traffic.txt")
-    if not os.path.exists(path):
-        return None
-    from fp8_block_scaled_group_b200 import build as pkg_build
+# The source files each kernel is built from; a recorded DRAM traffic figure
+# stays valid while their hash is unchanged.
+KERNEL_SOURCES = {
+    "gemm_blockscaled_kernel": ["gemm.cu", "group_quant.cuh", "ptx.cuh", "internal.h"],
+    "gemm_decode_kernel": ["gemm.cu", "group_quant.cuh", "ptx.cuh", "internal.h"],
+    "quant_act_multi_kernel": ["quant.cu", "group_quant.cuh", "ptx.cuh"],
+    "quant_act_single_kernel": ["quant.cu", "group_quant.cuh", "ptx.cuh"],
+    "silu_mul_quant_kernel": ["ffn.cu", "group_quant.cuh", "ptx.cuh"],
+}
+
+
+def kernel_digest(kernel: str) -> str:
     import hashlib
     h = hashlib.sha256()
-    for src in pkg_build.sources():
-        with open(src, "rb") as f:
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "fp8_block_scaled_group_b200", "csrc", name), "rb") as f:
             h.update(f.read())
-    digest = h.hexdigest()[:16]
+    return h.hexdigest()[:16]
+
+
+def read_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded from an ncu capture in profiles/traffic.txt,
+    or None when absent or when the kernel's sources changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path) or kernel not in KERNEL_SOURCES:
+        return None
+    digest = kernel_digest(kernel)
     with open(path) as f:
         for line in f:
             parts = line.split("#", 1)[0].split()
@@ -583,12 +597,14 @@ def ffn_arm(args):
     if m <= 64:
         gu_bytes = gemm_hbm_bytes(m, 2 * i, d)
         roofline = {"bound": "hbm", "kernel": "gemm_decode_kernel (gate|up)", "achieved": gu_bytes / (gu_ms * 1e-3) / 1e9,
-                    "peak": hbm, "unit": "GB/s", "frac": gu_bytes / (gu_ms * 1e-3) / 1e9 / hbm, "traffic": None,
+                    "peak": hbm, "unit": "GB/s", "frac": gu_bytes / (gu_ms * 1e-3) / 1e9 / hbm,
+                    "traffic": read_traffic("gemm_decode_kernel", args.workload),
                     "us": gu_ms * 1e3, "peak_source": f"{src} copy bandwidth"}
     else:
         tf = gu_flops / (gu_ms * 1e-3) / 1e12
         roofline = {"bound": "tensor", "kernel": "gemm_blockscaled_kernel (gate|up)", "achieved": tf,
-                    "peak": fp8_peak, "unit": "TFLOP/s", "frac": tf / fp8_peak, "traffic": None,
+                    "peak": fp8_peak, "unit": "TFLOP/s", "frac": tf / fp8_peak,
+                    "traffic": read_traffic("gemm_blockscaled_kernel", args.workload),
                     "us": gu_ms * 1e3, "peak_source": f"{src} bf16 burst x 2 (fp8:bf16 nominal ratio)"}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -608,7 +624,8 @@ def ffn_arm(args):
             "act_silu_mul_quant": {"bound": "hbm", "kernel": "silu_mul_quant_kernel",
                                    "achieved": act_bytes / (act_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
                                    "frac": act_bytes / (act_ms * 1e-3) / 1e9 / hbm, "us": act_ms * 1e3,
-                                   "bytes": act_bytes},
+                                   "bytes": act_bytes,
+                                   "traffic": read_traffic("silu_mul_quant_kernel", args.workload)},
             "cpu_baseline": cpu,
             "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": m * d * 2, "d2h_bytes_per_step": m * d * 2},
@@ -632,7 +649,13 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(FFN_WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-digests", action="store_true",
+                    help="print the source digest of each kernel (the key of profiles/traffic.txt) and exit")
     args = ap.parse_args()
+    if args.kernel_digests:
+        for kname in KERNEL_SOURCES:
+            print(kname, kernel_digest(kname))
+        return 0
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
     if args.workload in FFN_WORKLOADS:
         if args.impl == "reference":
