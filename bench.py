@@ -209,7 +209,7 @@ def sum_over_ranks(value: float, world: int) -> float:
 
 # ------------------------------------------------------------ CPU oracle --
 
-def cpu_oracle_sample(wl: dict, seed: int, target_s: float, threads: int):
+def cpu_oracle_sample(wl: dict, seed: int, target_s: float, threads: int, per_row: bool = False):
     """Time the oracle on a bounded sample of one step: quantize R rows of X and
     compute those R rows of the float64 reference output. Returns
     (TFLOP/s equivalent of 2*R*N*K / time, rows, seconds)."""
@@ -218,7 +218,8 @@ def cpu_oracle_sample(wl: dict, seed: int, target_s: float, threads: int):
     m, n, k = wl["m"], wl["n"], wl["k"]
     xb = inputs.activations(m, k, seed, wl["p"], wl["sigma"])
     wb = inputs.weights(n, k, wl["number"] + 1000)
-    wq, ws = oracle.quant_weight(wb)   # weight preparation is not part of the step
+    # weight preparation is not part of the step
+    wq, ws = oracle.quant_weight_rowwise(wb) if per_row else oracle.quant_weight(wb)
 
     def run(rows):
         t0 = time.perf_counter()
@@ -285,7 +286,7 @@ def ours_arm(args):
         wb = inputs.weights(n, k, seed_base + i)
         x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
         w = torch.from_numpy(wb.view(np.int16)).view(torch.bfloat16).to(dev)
-        wq, ws = api.quant_weight(w)
+        wq, ws = api.quant_weight_rowwise(w) if args.weight_format == "per_row" else api.quant_weight(w)
         del w
         work = torch.empty(api.linear_workspace_bytes(m, k), dtype=torch.uint8, device=dev)
         y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
@@ -293,9 +294,13 @@ def ours_arm(args):
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
+    linear_call = api.linear_decode_fused if args.decode_path == "fused" else api.linear
+    if args.decode_path == "fused" and m > 32:
+        raise SystemExit("--decode-path fused serves at most 32 tokens")
+
     def step(i):
         s = sets[i % N_SETS]
-        api.linear(s["x"], s["wq"], s["ws"], workspace=s["work"], out=s["y"])
+        linear_call(s["x"], s["wq"], s["ws"], workspace=s["work"], out=s["y"])
 
     for i in range(args.warmup):
         step(i)
@@ -381,7 +386,7 @@ def ours_arm(args):
     def e2e_step(i):
         s = sets[i % N_SETS]
         x_dev.copy_(x_host[i % N_SETS], non_blocking=True)
-        api.linear(x_dev, s["wq"], s["ws"], workspace=s["work"], out=s["y"])
+        linear_call(x_dev, s["wq"], s["ws"], workspace=s["work"], out=s["y"])
         y_host.copy_(s["y"], non_blocking=True)
 
     for i in range(args.warmup):
@@ -427,7 +432,8 @@ def ours_arm(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = os.cpu_count() or 1
-        v, rows, t = cpu_oracle_sample(wl, seed_base, args.cpu_seconds, threads)
+        v, rows, t = cpu_oracle_sample(wl, seed_base, args.cpu_seconds, threads,
+                                       per_row=args.weight_format == "per_row")
         cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": f"{rows} of {m} token rows of one step (quantize + float64 GEMM rows), "
                          f"{t:.1f} s, scaled to TFLOP/s"}
@@ -438,6 +444,7 @@ def ours_arm(args):
             "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
             "config": {"workload": args.workload, "m": m, "n": n, "k": k, "parallelism": f"replicas{world}",
+                       "weight_format": args.weight_format, "decode_path": args.decode_path,
                        "l2": f"{N_SETS} rotating input sets ({N_SETS * (m * k * 2 + n * k + m * n * 2) / 1e6:.0f} MB) > L2"},
             "roofline": roofline,
             "act_quant": {"bound": "hbm", "kernel": q_kernel, "achieved": quant_gbs, "peak": hbm, "unit": "GB/s",
@@ -460,7 +467,7 @@ def ours_arm(args):
 _FFN_ORACLE_W = {}
 
 
-def ffn_oracle_sample(wl: dict, threads: int):
+def ffn_oracle_sample(wl: dict, threads: int, target_s: float = 10.0):
     """Time the oracle's FFN on a bounded sample of one step's token rows;
     returns (TFLOP/s equivalent, rows, seconds). Weight preparation is not
     part of the step and is done once."""
@@ -473,10 +480,18 @@ def ffn_oracle_sample(wl: dict, threads: int):
         _FFN_ORACLE_W[key] = (*oracle.quant_weight(inputs.weights(2 * i, d, wl["seed"])),
                               *oracle.quant_weight(inputs.weights(d, i, wl["seed"] + 1)))
     wq_gu, ws_gu, wq_dn, ws_dn = _FFN_ORACLE_W[key]
+
+    def run(rows):
+        t0 = time.perf_counter()
+        oracle.ffn_ref(np.ascontiguousarray(xb[:rows]), wq_gu, ws_gu, wq_dn, ws_dn, threads=threads)
+        return time.perf_counter() - t0
+
     rows = max(1, min(m, threads))
-    t0 = time.perf_counter()
-    oracle.ffn_ref(np.ascontiguousarray(xb[:rows]), wq_gu, ws_gu, wq_dn, ws_dn, threads=threads)
-    t = time.perf_counter() - t0
+    t = run(rows)
+    if t < target_s and rows < m:
+        rows = int(min(m, max(rows, rows * target_s / max(t, 1e-3))))
+        rows = max(threads, rows - rows % threads) if rows >= threads else rows
+        t = run(rows)
     flops = 2.0 * rows * d * 2 * i + 2.0 * rows * i * d
     return flops / t / 1e12, rows, t
 
@@ -489,7 +504,7 @@ def ffn_reference_arm(args):
     vals = []
     rows = 0
     for j in range(args.warmup + args.steps):
-        v, rows, _ = ffn_oracle_sample(wl, threads)
+        v, rows, _ = ffn_oracle_sample(wl, threads, target_s=max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup))))
         if j >= args.warmup:
             vals.append(v)
     value = statistics.median(vals)
@@ -609,7 +624,7 @@ def ffn_arm(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = os.cpu_count() or 1
-        v, rows, t = ffn_oracle_sample(wl, threads)
+        v, rows, t = ffn_oracle_sample(wl, threads, target_s=args.cpu_seconds)
         cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": f"{rows} of {m} token rows of one FFN step, {t:.1f} s, scaled to TFLOP/s"}
     if rank == 0:
@@ -649,6 +664,10 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(FFN_WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--weight-format", choices=["block128", "per_row"], default="block128",
+                    help="weight scales per 128x128 block (the pages' format) or one per weight row")
+    ap.add_argument("--decode-path", choices=["two_launch", "fused"], default="two_launch",
+                    help="decode widths (M <= 32): quantizer + GEMM, or the GEMM with the quantizer fused in")
     ap.add_argument("--kernel-digests", action="store_true",
                     help="print the source digest of each kernel (the key of profiles/traffic.txt) and exit")
     args = ap.parse_args()
