@@ -21,8 +21,10 @@
 // per flop than a single-SM 128 x 256 tile. Per CTA, 12 warps:
 //   warp 0      TMA producer: A [128 x 128 B] and B [128 x 128 B] per K block
 //               into a 6-stage ring (128-byte swizzle), completion counted on
-//               the even CTA's barrier; plus the block's 128 activation
-//               scales (one K-major row slice) into an 8-slot local ring
+//               the even CTA's barrier; for long K also the block's 128
+//               activation scales (one K-major row slice) into an 8-slot
+//               local ring (otherwise the promotion warps load them, see
+//               kDirect below)
 //   warp 1      TMEM allocation for the pair; in the even CTA, the MMA issuer
 //               of the even K blocks (TMEM buffer 0)
 //   warp 2      in the even CTA, the MMA issuer of the odd K blocks (buffer 1)
@@ -111,10 +113,24 @@ __device__ __forceinline__ void spin_cycles(long long cycles) {
     }
 }
 
+// kDirect: where the promotion warps get the activation scales.
+//   true   each thread loads its row's scale of each K block from the
+//          K-major array in global memory (L2), four K blocks ahead; the
+//          TMA producer then issues only the A and B copies of a K block
+//   false  the TMA producer also copies the block's 128 scales of this
+//          CTA's rows into an 8-slot shared-memory ring
+// Measured on B200: with the producer doing one wait and two copies per K
+// block, M=1168 N=17408 K=5120 runs 6 % faster (137.5 -> 129.7 us); at
+// K=17408 the streaming operands evict the scales from L2 and the ring is
+// 10 % faster (488 vs 535 us). The host picks direct loads up to
+// kDirectScalesMaxG K blocks.
+constexpr uint32_t kDirectScalesMaxG = 64;
+
+template <bool kDirect>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                            const __grid_constant__ CUtensorMap tmS, const float* __restrict__ w_s,
-                            uint16_t* __restrict__ y, const Shape sh) {
+                            const __grid_constant__ CUtensorMap tmS, const float* __restrict__ s_k,
+                            const float* __restrict__ w_s, uint16_t* __restrict__ y, const Shape sh) {
     extern __shared__ uint8_t smem_raw[];
     GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t warp = threadIdx.x >> 5;
@@ -146,7 +162,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
-        tma_prefetch_desc(&tmS);
+        if (!kDirect) tma_prefetch_desc(&tmS);
     }
     if (warp == 1) {
         tmem_alloc_pair(&sm.tmem_base, kTmemCols);
@@ -176,14 +192,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 for (uint32_t kb = 0; kb < G; ++kb, ++it) {
                     const uint32_t s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
-                    const uint32_t ss = it % kScaleStages;
-                    const uint32_t sph = (it / kScaleStages) & 1u;
-                    if (!mbar_wait(&sm.empty[s], ph ^ 1u, abort) || !mbar_wait(&sm.sempty[ss], sph ^ 1u, abort)) {
+                    if (!mbar_wait(&sm.empty[s], ph ^ 1u, abort)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&sm.sfull[ss], kScaleBytes);
-                    tma_load_2d(sm.a_scale[ss], &tmS, &sm.sfull[ss], my_m, static_cast<int32_t>(kb));
+                    if constexpr (!kDirect) {
+                        const uint32_t ss = it % kScaleStages;
+                        const uint32_t sph = (it / kScaleStages) & 1u;
+                        if (!mbar_wait(&sm.sempty[ss], sph ^ 1u, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&sm.sfull[ss], kScaleBytes);
+                        tma_load_2d(sm.a_scale[ss], &tmS, &sm.sfull[ss], my_m, static_cast<int32_t>(kb));
+                    }
                     const uint32_t full_even = mapa_shared(smem_addr(&sm.full[s]), 0);
                     mbar_arrive_expect_tx_cluster(full_even, kTileBytesA + kTileBytesB);
                     tma_load_2d_pair(sm.a[s], &tmA, full_even, static_cast<int32_t>(kb * BK), my_m);
@@ -245,6 +267,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t r_local = quad * 32u + lane;
         const uint32_t tempty_even[2] = {mapa_shared(smem_addr(&sm.tempty[0]), 0),
                                          mapa_shared(smem_addr(&sm.tempty[1]), 0)};
+        // The activation scales come from the quantizer's K-major output.
+        if (kDirect) grid_dependency_wait();
         uint32_t it = 0;
         bool ok = true;
         for (uint32_t tile = pair; ok && tile < sh.num_tiles; tile += num_pairs) {
@@ -265,20 +289,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (uint32_t i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
             float w_next = per_row ? 1.0f : __ldg(ws_row);
+            // This row's activation scale of each K block, loaded four
+            // blocks ahead through a small register queue, so an L2 miss
+            // (the operands streaming through L2 can evict the scales at
+            // large K) stays off the K-block cycle. Rows past M have no
+            // scales and are never stored.
+            const float* a_row = s_k + (row_ok ? row : 0u);
+            float aq0 = 0.0f, aq1 = 0.0f, aq2 = 0.0f, aq3 = 0.0f;
+            if constexpr (kDirect) {
+                aq0 = row_ok && 0 < G ? __ldg(a_row) : 0.0f;
+                aq1 = row_ok && 1 < G ? __ldg(a_row + static_cast<size_t>(1) * sh.Mp) : 0.0f;
+                aq2 = row_ok && 2 < G ? __ldg(a_row + static_cast<size_t>(2) * sh.Mp) : 0.0f;
+                aq3 = row_ok && 3 < G ? __ldg(a_row + static_cast<size_t>(3) * sh.Mp) : 0.0f;
+            }
             for (uint32_t kb = 0; kb < G; ++kb, ++it) {
                 const uint32_t b = it & 1u;
                 const uint32_t tph = (it >> 1) & 1u;
                 const uint32_t ss = it % kScaleStages;
                 const uint32_t sph = (it / kScaleStages) & 1u;
                 const float w_cur = w_next;
+                float a_cur = aq0;
+                if constexpr (kDirect) {
+                    aq0 = aq1;
+                    aq1 = aq2;
+                    aq2 = aq3;
+                    aq3 = row_ok && kb + 4 < G ? __ldg(a_row + static_cast<size_t>(kb + 4) * sh.Mp) : 0.0f;
+                }
                 if (!per_row && kb + 1 < G) w_next = __ldg(ws_row + kb + 1);
-                const bool got = mbar_wait(&sm.sfull[ss], sph, abort) && mbar_wait(&sm.tfull[b], tph, abort);
+                const bool got = (kDirect || mbar_wait(&sm.sfull[ss], sph, abort)) && mbar_wait(&sm.tfull[b], tph, abort);
                 if (!__all_sync(0xFFFFFFFFu, got)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const float c = sm.a_scale[ss][r_local] * w_cur;
+                if constexpr (!kDirect) a_cur = sm.a_scale[ss][r_local];
+                const float c = a_cur * w_cur;
                 const float2 c2 = make_float2(c, c);
                 const uint32_t taddr = tmem + lane_off + b * BN + half * 128u;
 #pragma unroll
@@ -295,7 +340,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive_cluster(tempty_even[b]);
-                    mbar_arrive(&sm.sempty[ss]);
+                    if constexpr (!kDirect) mbar_arrive(&sm.sempty[ss]);
                 }
             }
             if (ok && row_ok && col_ok) {
@@ -340,9 +385,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 for (uint32_t it = from; it < issued; ++it)
                     if (it >= sm.consumed[it & 1u]) mbar_wait(&sm.full[it % kStages], (it / kStages) & 1u, &never);
             }
-            const uint32_t first = issued > kScaleStages ? issued - kScaleStages : 0u;
-            for (uint32_t it = first; it < issued; ++it)
-                mbar_wait(&sm.sfull[it % kScaleStages], (it / kScaleStages) & 1u, &never);
+            if constexpr (!kDirect) {
+                const uint32_t first = issued > kScaleStages ? issued - kScaleStages : 0u;
+                for (uint32_t it = first; it < issued; ++it)
+                    mbar_wait(&sm.sfull[it % kScaleStages], (it / kScaleStages) & 1u, &never);
+            }
             spin_cycles(200000);
         }
         __syncthreads();
@@ -761,15 +808,18 @@ const KernelSetup& setup_for_device() {
     KernelSetup& k = table[dev];
     if (!done[dev]) {
         done[dev] = true;
-        k.err = cudaFuncSetAttribute(gemm_blockscaled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(kSmemBytes));
-        cudaFuncAttributes attr;
-        if (k.err == cudaSuccess) k.err = cudaFuncGetAttributes(&attr, gemm_blockscaled_kernel);
         // setmaxnreg.inc waits until the registers it asks for are free in
         // the CTA's allocation: refuse to launch a build whose allocation
         // cannot cover the split.
-        if (k.err == cudaSuccess && static_cast<uint32_t>(attr.numRegs) < kLaunchRegsNeeded)
-            k.err = cudaErrorInvalidConfiguration;
+        for (auto fn : {gemm_blockscaled_kernel<true>, gemm_blockscaled_kernel<false>}) {
+            if (k.err == cudaSuccess)
+                k.err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kSmemBytes));
+            cudaFuncAttributes attr;
+            if (k.err == cudaSuccess) k.err = cudaFuncGetAttributes(&attr, fn);
+            if (k.err == cudaSuccess && static_cast<uint32_t>(attr.numRegs) < kLaunchRegsNeeded)
+                k.err = cudaErrorInvalidConfiguration;
+        }
         if (k.err == cudaSuccess) k.err = cudaDeviceGetAttribute(&k.sms, cudaDevAttrMultiProcessorCount, dev);
     }
     return k;
@@ -887,8 +937,11 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = L.pdl ? 1 : 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel, ta, tb, ts, L.w_scale,
-                                       static_cast<uint16_t*>(L.y), sh);
+    const bool direct = sh.G <= kDirectScalesMaxG;
+    cudaError_t e = direct ? cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<true>, ta, tb, ts, L.s_k, L.w_scale,
+                                                static_cast<uint16_t*>(L.y), sh)
+                           : cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<false>, ta, tb, ts, L.s_k, L.w_scale,
+                                                static_cast<uint16_t*>(L.y), sh);
     note_launch();
     return e != cudaSuccess ? e : cudaGetLastError();
 }
