@@ -34,7 +34,10 @@
 //               columns, one weight block), one row per thread
 // Tiles are visited M-fastest so the pairs running at one time share weight
 // tiles through L2. Rows past M and columns past N are zero-filled by TMA
-// and never stored.
+// and never stored. With per-row weight scales (one per weight row, the
+// scale block 1 x K of `dequant_fp8_bf16_into`'s per-row layout) the
+// promotion folds in a_s[t][g] only and the epilogue multiplies each output
+// column by its row's scale once.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
