@@ -187,24 +187,36 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(value: float, world: int) -> float:
+def max_over_ranks(value: float, world: int, device: str = "cuda") -> float:
+    """The largest value over all ranks (the job's time is its slowest rank's)."""
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def sum_over_ranks(value: float, world: int) -> float:
+def sum_over_ranks(value: float, world: int, device: str = "cuda") -> float:
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def rank_input_seed(seed_base: int, rank: int, set_index: int) -> int:
+    """Seed of input set `set_index` on `rank`: every rank draws its own tokens."""
+    return seed_base + 7919 * (rank * N_SETS + set_index)
+
+
+def weak_scaling_value(units_per_rank_step: float, world: int, steps: int, ms_total: float) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest
+    rank's time (units per second)."""
+    return units_per_rank_step * world * steps / (ms_total * 1e-3)
 
 
 # ------------------------------------------------------------ CPU oracle --
@@ -282,7 +294,7 @@ def ours_arm(args):
     # Input sets: each rank draws its own tokens (weak scaling).
     sets = []
     for i in range(N_SETS):
-        xb = inputs.activations(m, k, seed_base + 7919 * (rank * N_SETS + i), wl["p"], wl["sigma"])
+        xb = inputs.activations(m, k, rank_input_seed(seed_base, rank, i), wl["p"], wl["sigma"])
         wb = inputs.weights(n, k, seed_base + i)
         x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(dev)
         w = torch.from_numpy(wb.view(np.int16)).view(torch.bfloat16).to(dev)
@@ -403,8 +415,8 @@ def ours_arm(args):
     e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world)
 
     flops = 2.0 * m * n * k
-    value = flops * world * args.steps / (ms_total * 1e-3) / 1e12
-    e2e_value = flops * world * args.steps / (e2e_ms * 1e-3) / 1e12
+    value = weak_scaling_value(flops, world, args.steps, ms_total) / 1e12
+    e2e_value = weak_scaling_value(flops, world, args.steps, e2e_ms) / 1e12
     hbm, bf16, bf16_sus, src = load_peaks()
     fp8_peak = bf16 * 2.0  # fp8 dense = 2x bf16 dense (nominal 4.5 / 2.25 PF)
     gemm_us = statistics.mean(g_ms) * 1e3
@@ -535,7 +547,7 @@ def ffn_arm(args):
     m, d, i = wl["m"], wl["d"], wl["i"]
     sets = []
     for j in range(N_SETS):
-        xb = inputs.activations(m, d, wl["seed"] + 7919 * (rank * N_SETS + j))
+        xb = inputs.activations(m, d, rank_input_seed(wl["seed"], rank, j))
         to_dev = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
         wgu, wsgu = api.quant_weight(to_dev(inputs.weights(2 * i, d, wl["seed"] + 2 * j)))
         wdn, wsdn = api.quant_weight(to_dev(inputs.weights(d, i, wl["seed"] + 2 * j + 1)))
@@ -629,7 +641,7 @@ def ffn_arm(args):
                "sample": f"{rows} of {m} token rows of one FFN step, {t:.1f} s, scaled to TFLOP/s"}
     if rank == 0:
         line = {
-            "metric": FFN_METRIC, "value": flops * world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "metric": FFN_METRIC, "value": weak_scaling_value(flops, world, 1, ms) / 1e12, "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
             "data": "synthetic",
@@ -642,7 +654,7 @@ def ffn_arm(args):
                                    "bytes": act_bytes,
                                    "traffic": read_traffic("silu_mul_quant_kernel", args.workload)},
             "cpu_baseline": cpu,
-            "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": weak_scaling_value(flops, world, 1, e2e_ms) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": m * d * 2, "d2h_bytes_per_step": m * d * 2},
             "gpu_launches": int(sum_over_ranks(launches, world)),
             "clocks": clk,
