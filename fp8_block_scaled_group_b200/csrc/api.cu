@@ -278,7 +278,6 @@ fp8q_status fp8q_linear_ex(const void* x, const void* wq, const float* w_scale, 
     fp8q_status st = check_quant_args(x, ws, nullptr, s_k, m, k);
     if (st != FP8Q_OK) return st;
     if ((st = check_gemm_args(ws, s_k, wq, w_scale, y, m, n, k)) != FP8Q_OK) return st;
-    if (m == 0) return FP8Q_OK;
     const bool per_row = weight_format == FP8Q_WEIGHT_PER_ROW;
     if ((st = fp8q_quant_act(x, ws, nullptr, s_k, m, k, stream)) != FP8Q_OK) return st;
     // The GEMM is the quantizer's programmatic dependent: its set-up (barriers,
@@ -361,6 +360,9 @@ fp8q_status fp8q_ffn(const void* x, const void* w_gate_up, const float* w_gate_u
     if (st != FP8Q_OK) return st;
     if (m == 0) return FP8Q_OK;
     if (!x || !w_gate_up || !w_gate_up_scale || !w_down || !w_down_scale || !y || !workspace) return FP8Q_ERR_NULL;
+    // gate|up is [m, 2i]: the stacked width and the element count must stay
+    // below 2^31 like every other operand (2i is formed in 32 bits below)
+    if (static_cast<uint64_t>(m) * 2u * i >= (1ull << 31)) return FP8Q_ERR_SHAPE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < off[5]) return FP8Q_ERR_WORKSPACE;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     void* q_x = ws + off[0];

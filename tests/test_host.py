@@ -208,6 +208,10 @@ def test_silu_mul_quant_and_ffn_argument_errors():
     assert lib.fp8q_ffn(A, B, C, D, E, A, ws, need - 1, m, d, i, None) == 4
     assert lib.fp8q_ffn(A, B, C, D, E, A, ctypes.c_void_p(0x1000010), need, m, d, i, None) == 4
     assert lib.fp8q_ffn(A, B, C, D, ODD, A, ws, need, m, d, i, None) == 3
+    # gate|up [m, 2i] past 2^31 elements, and a 2i that would wrap in 32 bits
+    big_i = 1 << 30
+    assert lib.fp8q_ffn(A, B, C, D, E, A, ws, 1 << 62, 2, d, big_i, None) == 2
+    assert lib.fp8q_ffn(A, B, C, D, E, A, ws, 1 << 62, 1, d, (1 << 31) + 128, None) == 2
 
 
 def test_ffn_workspace_layout():
