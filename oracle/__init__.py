@@ -4,7 +4,9 @@ A ctypes wrapper around ``fp8q_oracle.c``: the plain, slow CPU restatement of
 per-token-group FP8 activation quantization, 128x128 block weight
 quantization, the float64 dequantized GEMM reference, and the dense FFN built
 from them: SiLU(gate) * up rounded to bf16 and quantized again for the down
-projection (pages
+projection, the FP8-to-bf16 weight dequantizer, and the NVFP4 projection
+arms: E2M1 elements packed two to a byte with E4M3 scales per 16 along K and
+an fp32 second-level scale (pages
 "spark_model/layers/ops/dispatch_proj.rs" and
 "spark_model/layers/ops/fp8_act_quant_floor.rs").
 
@@ -85,6 +87,21 @@ def _load():
         lib.oracle_round_bf16_array.restype = None
         lib.oracle_silu_mul_quant.argtypes = [P, P, ctypes.c_size_t, U32, U32, P, P, P]
         lib.oracle_silu_mul_quant.restype = ctypes.c_int
+        lib.oracle_dequant_fp8_bf16.argtypes = [P, P, U32, U32, U32, U32, P]
+        lib.oracle_dequant_fp8_bf16.restype = ctypes.c_int
+        lib.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e2m1_decode.restype = ctypes.c_double
+        lib.oracle_e2m1_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e2m1_encode.restype = ctypes.c_uint8
+        lib.oracle_e2m1_encode_array.argtypes = [P, ctypes.c_size_t, P]
+        lib.oracle_e2m1_encode_array.restype = None
+        lib.oracle_nvfp4_quant.argtypes = [P, U32, U32, ctypes.c_float, P, P]
+        lib.oracle_nvfp4_quant.restype = ctypes.c_int
+        lib.oracle_nvfp4_global_scale.argtypes = [P, ctypes.c_size_t]
+        lib.oracle_nvfp4_global_scale.restype = ctypes.c_float
+        lib.oracle_nvfp4_gemm_ref_rows.argtypes = [P, P, ctypes.c_float, P, P, ctypes.c_float, U32, U32, P,
+                                                   ctypes.c_size_t, ctypes.c_size_t, P]
+        lib.oracle_nvfp4_gemm_ref_rows.restype = None
         _lib = lib
         return lib
 
@@ -268,3 +285,90 @@ def ffn_ref(x_bf16: np.ndarray, wq_gate_up: np.ndarray, ws_gate_up: np.ndarray,
     y = gemm_ref(q_h, s_h, wq_down, ws_down, threads=threads)
     return {"q_x": q_x, "s_x": s_x, "gate": gate, "up": up,
             "q_h": q_h, "s_h": s_h, "s_h_kmajor": s_h_k, "y": y}
+
+
+# ------------------------------------------------ FP8 weight back to bf16 --
+
+def dequant_fp8_bf16(wq: np.ndarray, w_scale: np.ndarray) -> np.ndarray:
+    """e4m3 codes [N,K] and their fp32 scales -> bf16 bits [N,K], each the
+    bf16 nearest to code * scale. The scale's shape selects the geometry:
+    [N/128, K/128] (128x128 blocks) or [N] (one per row)."""
+    wq = np.ascontiguousarray(wq, dtype=np.uint8)
+    ws = np.ascontiguousarray(w_scale, dtype=np.float32)
+    n, k = wq.shape
+    if ws.shape == (n,):
+        block_n, block_k = 1, k
+    else:
+        assert ws.shape == (n // GROUP, k // GROUP)
+        block_n, block_k = GROUP, GROUP
+    out = np.empty((n, k), np.uint16)
+    rc = _load().oracle_dequant_fp8_bf16(_ptr(wq), _ptr(ws), n, k, block_n, block_k, _ptr(out))
+    assert rc == 0
+    return out
+
+
+# ---------------------------------------------------------------- NVFP4 --
+
+NVFP4_BLOCK = 16
+
+
+def e2m1_decode(code: int) -> float:
+    return float(_load().oracle_e2m1_decode(int(code)))
+
+
+def e2m1_encode(t: float) -> int:
+    return int(_load().oracle_e2m1_encode(float(t)))
+
+
+def e2m1_encode_array(t: np.ndarray) -> np.ndarray:
+    """Encode each fp32 value with the scalar E2M1 encoder (for sweeps)."""
+    t = np.ascontiguousarray(t, dtype=np.float32).ravel()
+    out = np.empty(t.size, np.uint8)
+    _load().oracle_e2m1_encode_array(_ptr(t), t.size, _ptr(out))
+    return out
+
+
+def nvfp4_quant(x_bf16: np.ndarray, s2: float = 1.0):
+    """bf16 bits [R,K] -> (q [R,K/2] u8, two E2M1 codes a byte with the even
+    K index in the low nibble; sf [R,K/16] u8 E4M3 block scales), packed with
+    second-level scale s2."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    r, k = x.shape
+    if k % NVFP4_BLOCK:
+        raise ValueError("k must be a multiple of 16")
+    q = np.empty((r, k // 2), np.uint8)
+    sf = np.empty((r, k // NVFP4_BLOCK), np.uint8)
+    rc = _load().oracle_nvfp4_quant(_ptr(x), r, k, float(s2), _ptr(q), _ptr(sf))
+    if rc != 0:
+        raise ValueError("s2 must be a positive, finite fp32 value")
+    return q, sf
+
+
+def nvfp4_global_scale(x_bf16: np.ndarray) -> float:
+    """max(amax, 1e-10) / 2688 in fp32: the second-level scale of a synthetic
+    NVFP4 checkpoint weight."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    return float(_load().oracle_nvfp4_global_scale(_ptr(x), x.size))
+
+
+def nvfp4_gemm_ref(qa: np.ndarray, sfa: np.ndarray, s2a: float, qw: np.ndarray, sfw: np.ndarray,
+                   s2w: float, rows: np.ndarray | None = None) -> np.ndarray:
+    """Float64 reference Y[rows, N] of the NVFP4 projection, operands as
+    nvfp4_quant returns them."""
+    qa = np.ascontiguousarray(qa, dtype=np.uint8)
+    sfa = np.ascontiguousarray(sfa, dtype=np.uint8)
+    qw = np.ascontiguousarray(qw, dtype=np.uint8)
+    sfw = np.ascontiguousarray(sfw, dtype=np.uint8)
+    m, half_k = qa.shape
+    k = 2 * half_k
+    n = qw.shape[0]
+    assert qw.shape == (n, half_k) and sfa.shape == (m, k // NVFP4_BLOCK) and sfw.shape == (n, k // NVFP4_BLOCK)
+    if rows is None:
+        rows_arr = np.arange(m, dtype=np.int64)
+    else:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        assert rows_arr.size == 0 or (rows_arr.min() >= 0 and rows_arr.max() < m)
+    ref = np.empty((rows_arr.size, n), np.float64)
+    _load().oracle_nvfp4_gemm_ref_rows(_ptr(qa), _ptr(sfa), float(s2a), _ptr(qw), _ptr(sfw), float(s2w),
+                                       n, k, _ptr(rows_arr), 0, rows_arr.size, _ptr(ref))
+    return ref

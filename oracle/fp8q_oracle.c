@@ -25,6 +25,11 @@
  * scales); the code decision is taken on that fp32 quotient. The encoder
  * works in double, where every step below is exact.
  *
+ * Beyond the FP8 linear it restates the dense FFN's SiLU(gate) * up step,
+ * the per-row weight format, the FP8-to-bf16 weight dequantizer and the
+ * NVFP4 projection arms (E2M1 elements with E4M3 scales per 16 along K);
+ * each section states its own reading of the pages.
+ *
  * Build: gcc -O2 -std=c11 -fPIC -shared (no -ffast-math, no -ffp-contract
  * beyond "off": fp32 results must be IEEE single-rounded).
  */
@@ -502,4 +507,211 @@ void oracle_silu_mul_bf16_array(const uint16_t *g, const uint16_t *u, size_t cou
     size_t i;
     for (i = 0; i < count; i++)
         h[i] = oracle_silu_mul_bf16(g[i], u[i]);
+}
+
+/* --------------------------------------------- FP8 weight back to bf16 -- */
+
+/*
+ * Dequantize an FP8 weight to bf16 (dispatch_proj.rs, `dequant_fp8_bf16_into`:
+ * an [N,K] bf16 result, block (128,128) or, for the per-row format,
+ * (1,K)). The pages do not print the kernel; the reading taken is the plain
+ * one: each element is the bf16 nearest to the exact product
+ *   deq(wq[r][c]) * w_s[(r/block_n) * (k/block_k) + c/block_k]
+ * (ties to even, sign of zero kept). The product of a 4-bit and a 24-bit
+ * significand is exact in double, so there is one rounding.
+ * Returns 0, or -1 if the blocks do not tile [n, k].
+ */
+int oracle_dequant_fp8_bf16(const uint8_t *wq, const float *w_s, uint32_t n, uint32_t k,
+                            uint32_t block_n, uint32_t block_k, uint16_t *out)
+{
+    uint32_t r, c, sk;
+    if (block_n == 0 || block_k == 0 || n % block_n || k % block_k)
+        return -1;
+    sk = k / block_k;
+    for (r = 0; r < n; r++) {
+        for (c = 0; c < k; c++) {
+            double v = oracle_e4m3_decode(wq[(size_t)r * k + c]) *
+                       (double)w_s[(size_t)(r / block_n) * sk + c / block_k];
+            uint16_t sign = signbit(v) ? 0x8000u : 0u;
+            out[(size_t)r * k + c] =
+                v == 0.0 ? sign : (uint16_t)(sign | bf16_magnitude_bits(fabsl((long double)v), 0));
+        }
+    }
+    return 0;
+}
+
+/* --------------------------------------------------------------- NVFP4 -- */
+
+/*
+ * The NVFP4 projection arms (dispatch_proj.rs, doc comments of
+ * `cutlass_nvfp4_proj`, `cutlass_nvfp4_weight_transposed_cached` and
+ * `cutlass_nvfp4_proj_from_fp8`). The pages fix the geometry: two 4-bit
+ * elements per byte along K ([K/2, N] data), one scale per 16 elements along
+ * K ([K/16, N] scales) and one fp32 second-level scale per weight
+ * (`weight_scale_2`; 1.0 for a weight packed from an FP8 checkpoint). They
+ * print neither the element format nor the packer. The readings taken:
+ *   - elements are NVFP4's E2M1 (1 sign bit, 2 exponent bits with bias 1,
+ *     1 mantissa bit; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6; no Inf, no NaN)
+ *     and block scales are E4M3 codes, the format's own definition;
+ *   - within a byte the element with the even K index sits in the low nibble;
+ *   - the packer follows the format's plain recipe, one fp32 operation a step:
+ *       amax = max_j |x_j|                    over 16 consecutive K elements
+ *       sf   = e4m3_rne_satfinite(amax / (6 * s2))
+ *       s    = deq(sf) * s2                   the block's effective scale
+ *       q_j  = e2m1_rne_satfinite(x_j / s)    (s == 0: every q_j is a zero
+ *                                              carrying the sign of x_j)
+ *     with s2 the second-level scale of the operand.
+ */
+
+#define NVFP4_BLOCK 16       /* K elements that share one block scale */
+#define E2M1_MAX 6.0         /* largest E2M1 magnitude */
+
+/* Decode one E2M1 code (low 4 bits of `code`). Exponent field 0 holds the
+   subnormals m * 0.5; otherwise the value is 2^(e-1) * (1 + m/2). */
+double oracle_e2m1_decode(uint8_t code)
+{
+    int sign = (code >> 3) & 1;
+    int e = (code >> 1) & 3;
+    int m = code & 1;
+    double mag = (e == 0) ? 0.5 * (double)m : ldexp(1.0 + 0.5 * (double)m, e - 1);
+    return sign ? -mag : mag;
+}
+
+/*
+ * Encode one fp32 value into E2M1, round to nearest with ties to the even
+ * code, saturating at 6 and keeping the sign of zero. Inside a binade the
+ * representable magnitudes are evenly spaced (0.5 below 2, 1 in [2, 4),
+ * 2 in [4, 6]); a/spacing is then an integer whose parity is the parity of
+ * the code, so rounding that quotient half-to-even rounds the code
+ * half-to-even. NaN input is outside the contract.
+ */
+uint8_t oracle_e2m1_encode(float t)
+{
+    uint8_t sign = signbit(t) ? 0x8 : 0x0;
+    double a = fabs((double)t);
+    double spacing, r;
+    uint8_t c;
+    if (a >= E2M1_MAX)
+        return (uint8_t)(sign | 0x7);
+    spacing = a < 2.0 ? 0.5 : (a < 4.0 ? 1.0 : 2.0);
+    r = round_half_even(a / spacing) * spacing;   /* exact: spacing is a power of two */
+    for (c = 0; c < 8; c++)
+        if (oracle_e2m1_decode(c) == r)
+            return (uint8_t)(sign | c);
+    return 0xFF; /* unreachable: r is always one of the eight magnitudes */
+}
+
+/* Encode `count` fp32 values one by one with oracle_e2m1_encode (sweeps). */
+void oracle_e2m1_encode_array(const float *t, size_t count, uint8_t *out)
+{
+    size_t i;
+    for (i = 0; i < count; i++)
+        out[i] = oracle_e2m1_encode(t[i]);
+}
+
+/*
+ * Pack a bf16 matrix into NVFP4 along K with second-level scale s2:
+ *   x   bf16 bits [r, k] row-major
+ *   q   [r, k/2] bytes: element 2j of a row in the low nibble of byte j,
+ *       element 2j+1 in the high nibble
+ *   sf  E4M3 codes [r, k/16] row-major, one per 16-element block
+ * Returns 0, or -1 if k is not a multiple of 16 or s2 is not a positive,
+ * finite fp32 value.
+ */
+int oracle_nvfp4_quant(const uint16_t *x, uint32_t r, uint32_t k, float s2, uint8_t *q, uint8_t *sf)
+{
+    uint32_t row, b, j, nb;
+    if (k % NVFP4_BLOCK != 0 || !(s2 > 0.0f) || isinf(s2))
+        return -1;
+    nb = k / NVFP4_BLOCK;
+    for (row = 0; row < r; row++) {
+        for (b = 0; b < nb; b++) {
+            float v[NVFP4_BLOCK];
+            float amax = 0.0f, t, s;
+            uint8_t code;
+            for (j = 0; j < NVFP4_BLOCK; j++) {
+                v[j] = oracle_bf16_to_f32(x[(size_t)row * k + (size_t)b * NVFP4_BLOCK + j]);
+                if (fabsf(v[j]) > amax)
+                    amax = fabsf(v[j]);
+            }
+            t = amax / (6.0f * s2);                       /* fp32 product, then fp32 division */
+            code = oracle_e4m3_encode(t);
+            s = (float)oracle_e4m3_decode(code) * s2;     /* one fp32 product */
+            sf[(size_t)row * nb + b] = code;
+            for (j = 0; j < NVFP4_BLOCK; j += 2) {
+                uint8_t lo, hi;
+                if (s == 0.0f) {
+                    lo = signbit(v[j]) ? 0x8 : 0x0;
+                    hi = signbit(v[j + 1]) ? 0x8 : 0x0;
+                } else {
+                    lo = oracle_e2m1_encode(v[j] / s);    /* one fp32 division */
+                    hi = oracle_e2m1_encode(v[j + 1] / s);
+                }
+                q[((size_t)row * k + (size_t)b * NVFP4_BLOCK + j) / 2] = (uint8_t)(lo | (hi << 4));
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * The second-level scale of a synthetic NVFP4 checkpoint weight: the pages
+ * take `weight_scale_2` from the checkpoint and never say how it was made.
+ * The reading taken is the format's usual choice, which lets the largest
+ * block scale reach E4M3's 448:
+ *   s2 = max(amax over the whole tensor, 1e-10) / (6 * 448)
+ * (one fp32 division; 2688 is exact).
+ */
+float oracle_nvfp4_global_scale(const uint16_t *x, size_t count)
+{
+    float amax = 0.0f;
+    size_t i;
+    for (i = 0; i < count; i++) {
+        float v = fabsf(oracle_bf16_to_f32(x[i]));
+        if (v > amax)
+            amax = v;
+    }
+    return (amax > 1e-10f ? amax : 1e-10f) / 2688.0f;
+}
+
+/*
+ * Float64 reference of the NVFP4 projection for the requested rows:
+ *   ref[i][col] = s2a * s2w * sum_kk deq(qa[r_i][kk]) * deq(sfa[r_i][kk/16])
+ *                                  * deq(qw[col][kk]) * deq(sfw[col][kk/16])
+ *   qa, sfa  packed activation [m, k/2] and its E4M3 scales [m, k/16]
+ *   qw, sfw  packed weight [n, k/2] and its E4M3 scales [n, k/16]
+ * (layouts as oracle_nvfp4_quant writes them); ref float64 [rows, n].
+ * Every product and every 16-element partial sum is exact in double.
+ */
+void oracle_nvfp4_gemm_ref_rows(const uint8_t *qa, const uint8_t *sfa, float s2a,
+                                const uint8_t *qw, const uint8_t *sfw, float s2w,
+                                uint32_t n, uint32_t k, const int64_t *rows,
+                                size_t first, size_t count, double *ref)
+{
+    double e2m1[16], e4m3[256];
+    uint32_t nb = k / NVFP4_BLOCK, col, b, j;
+    size_t i;
+    for (i = 0; i < 16; i++)
+        e2m1[i] = oracle_e2m1_decode((uint8_t)i);
+    for (i = 0; i < 256; i++)
+        e4m3[i] = oracle_e4m3_decode((uint8_t)i);
+    for (i = first; i < first + count; i++) {
+        int64_t r = rows ? rows[i] : (int64_t)i;
+        for (col = 0; col < n; col++) {
+            double acc = 0.0;
+            for (b = 0; b < nb; b++) {
+                double part = 0.0;
+                for (j = 0; j < NVFP4_BLOCK; j++) {
+                    size_t kk = (size_t)b * NVFP4_BLOCK + j;
+                    uint8_t ba = qa[((size_t)r * k + kk) / 2];
+                    uint8_t bw = qw[((size_t)col * k + kk) / 2];
+                    uint8_t ca = (kk & 1) ? (uint8_t)(ba >> 4) : (uint8_t)(ba & 0xF);
+                    uint8_t cw = (kk & 1) ? (uint8_t)(bw >> 4) : (uint8_t)(bw & 0xF);
+                    part += e2m1[ca] * e2m1[cw];
+                }
+                acc += part * e4m3[sfa[(size_t)r * nb + b]] * e4m3[sfw[(size_t)col * nb + b]];
+            }
+            ref[i * n + col] = acc * (double)s2a * (double)s2w;
+        }
+    }
 }
