@@ -59,6 +59,13 @@ SIGNATURES = {
     "fp8q_ffn_workspace_bytes": (SZ, [U32, U32, U32]),
     "fp8q_ffn": (ctypes.c_int, [P, P, P, P, P, P, P, SZ, U32, U32, U32, P]),
     "fp8q_check_silu_mul": (ctypes.c_int, [P, P, P]),
+    "fp8q_nvfp4_sf_mma_bytes": (SZ, [U32, U32]),
+    "fp8q_nvfp4_quant": (ctypes.c_int, [P, P, P, P, ctypes.c_float, U32, U32, P]),
+    "fp8q_nvfp4_gemm": (ctypes.c_int, [P, P, ctypes.c_float, P, P, ctypes.c_float, P, U32, U32, U32, P]),
+    "fp8q_nvfp4_linear_workspace_bytes": (SZ, [U32, U32]),
+    "fp8q_nvfp4_linear": (ctypes.c_int, [P, ctypes.c_float, P, P, ctypes.c_float, P, P, SZ, U32, U32, U32, P]),
+    "fp8q_dequant_fp8_bf16": (ctypes.c_int, [P, P, I32, P, U32, U32, P]),
+    "fp8q_convert_e2m1": (ctypes.c_int, [P, P, SZ, P]),
     "fp8q_convert_e4m3": (ctypes.c_int, [P, P, SZ, P]),
     "fp8q_check_division": (ctypes.c_int, [P, P]),
     "fp8q_launch_count": (ctypes.c_uint64, []),

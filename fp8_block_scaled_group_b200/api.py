@@ -250,6 +250,88 @@ def linear_decode_fused(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor
     return y
 
 
+# ---------------------------------------------------------------- NVFP4 --
+
+NVFP4_BLOCK = 16
+
+
+def nvfp4_sf_mma_bytes(rows: int, k: int) -> int:
+    return int(_lib.load().fp8q_nvfp4_sf_mma_bytes(rows, k))
+
+
+def nvfp4_quant(x: torch.Tensor, s2: float = 1.0, row_major: bool = True, stream=None):
+    """x bf16 [R, K] -> (q uint8 [R, K/2] packed E2M1, sf_row uint8 [R, K/16] E4M3
+    or None, sf_mma uint8 [nvfp4_sf_mma_bytes(R, K)] in the MMA layout)."""
+    r, k = x.shape
+    _need(x, torch.bfloat16, (r, k), "x")
+    q = torch.empty((r, k // 2), dtype=torch.uint8, device=x.device)
+    sf_row = torch.empty((r, k // NVFP4_BLOCK), dtype=torch.uint8, device=x.device) if row_major else None
+    sf_mma = torch.empty((nvfp4_sf_mma_bytes(r, k),), dtype=torch.uint8, device=x.device)
+    _lib.check(_lib.load().fp8q_nvfp4_quant(_p(x), _p(q), _p(sf_row), _p(sf_mma), float(s2), r, k,
+                                             _stream(stream)), "fp8q_nvfp4_quant")
+    return q, sf_row, sf_mma
+
+
+def nvfp4_gemm(qa: torch.Tensor, sfa_mma: torch.Tensor, s2a: float, qw: torch.Tensor, sfw_mma: torch.Tensor,
+               s2w: float, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """qa uint8 [M, K/2] + MMA-layout scales, qw uint8 [N, K/2] + MMA-layout scales -> y bf16 [M, N]."""
+    m, half_k = qa.shape
+    k = 2 * half_k
+    n = qw.shape[0]
+    _need(qa, torch.uint8, (m, half_k), "qa")
+    _need(qw, torch.uint8, (n, half_k), "qw")
+    _need(sfa_mma, torch.uint8, (nvfp4_sf_mma_bytes(m, k),), "sfa_mma")
+    _need(sfw_mma, torch.uint8, (nvfp4_sf_mma_bytes(n, k),), "sfw_mma")
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=qa.device) if out is None else out
+    _need(y, torch.bfloat16, (m, n), "y")
+    _lib.check(_lib.load().fp8q_nvfp4_gemm(_p(qa), _p(sfa_mma), float(s2a), _p(qw), _p(sfw_mma), float(s2w),
+                                            _p(y), m, n, k, _stream(stream)), "fp8q_nvfp4_gemm")
+    return y
+
+
+def nvfp4_linear_workspace_bytes(m: int, k: int) -> int:
+    return int(_lib.load().fp8q_nvfp4_linear_workspace_bytes(m, k))
+
+
+def nvfp4_linear(x: torch.Tensor, qw: torch.Tensor, sfw_mma: torch.Tensor, s2w: float, s2a: float = 1.0,
+                 workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                 stream=None) -> torch.Tensor:
+    """NVFP4 projection: x bf16 [M, K] packed inside the call, times the packed weight -> y bf16 [M, N]."""
+    m, k = x.shape
+    n = qw.shape[0]
+    _need(x, torch.bfloat16, (m, k), "x")
+    _need(qw, torch.uint8, (n, k // 2), "qw")
+    _need(sfw_mma, torch.uint8, (nvfp4_sf_mma_bytes(n, k),), "sfw_mma")
+    if workspace is None:
+        workspace = torch.empty(nvfp4_linear_workspace_bytes(m, k), dtype=torch.uint8, device=x.device)
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _need(y, torch.bfloat16, (m, n), "y")
+    _lib.check(_lib.load().fp8q_nvfp4_linear(_p(x), float(s2a), _p(qw), _p(sfw_mma), float(s2w), _p(y),
+                                              _p(workspace), workspace.numel(), m, n, k, _stream(stream)),
+               "fp8q_nvfp4_linear")
+    return y
+
+
+def dequant_fp8_bf16(wq: torch.Tensor, w_scale: torch.Tensor, stream=None) -> torch.Tensor:
+    """wq uint8 [N, K] with fp32 scales [N/128, K/128] or [N] -> bf16 [N, K]."""
+    n, k = wq.shape
+    _need(wq, torch.uint8, (n, k), "wq")
+    fmt = _weight_format(w_scale, n, k)
+    y = torch.empty((n, k), dtype=torch.bfloat16, device=wq.device)
+    _lib.check(_lib.load().fp8q_dequant_fp8_bf16(_p(wq), _p(w_scale), fmt, _p(y), n, k, _stream(stream)),
+               "fp8q_dequant_fp8_bf16")
+    return y
+
+
+def convert_e2m1(t: torch.Tensor, stream=None) -> torch.Tensor:
+    """fp32 CUDA tensor -> uint8 E2M1 codes (one per byte) with the packer's conversion."""
+    if not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+        raise ValueError("t must be a contiguous fp32 CUDA tensor")
+    out = torch.empty(t.shape, dtype=torch.uint8, device=t.device)
+    _lib.check(_lib.load().fp8q_convert_e2m1(_p(t), _p(out), t.numel(), _stream(stream)), "fp8q_convert_e2m1")
+    return out
+
+
 def convert_e4m3(t: torch.Tensor, stream=None) -> torch.Tensor:
     """fp32 CUDA tensor -> uint8 e4m3 codes with the quantizers' conversion."""
     if not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():

@@ -9,6 +9,7 @@
 
 #include "fp8q.h"
 #include "internal.h"
+#include "nvfp4.h"
 
 namespace fp8q {
 
@@ -397,6 +398,107 @@ fp8q_status fp8q_check_silu_mul(unsigned long long* counts, uint32_t* max_err_bi
     return from_cuda(launch_check_silu_mul(counts, max_err_bits, static_cast<cudaStream_t>(stream)));
 }
 
+// ---------------------------------------------------------------- NVFP4 --
+
+size_t fp8q_nvfp4_sf_mma_bytes(uint32_t rows, uint32_t k) { return nvfp4_sf_mma_bytes(rows, k); }
+
+fp8q_status fp8q_nvfp4_quant(const void* x, void* q, void* sf_rowmajor, void* sf_mma, float s2, uint32_t rows,
+                             uint32_t k, void* stream) {
+    if (k == 0 || k % 64u) return FP8Q_ERR_SHAPE;
+    if (!(s2 > 0.0f) || std::isinf(s2)) return FP8Q_ERR_ARG;
+    if (rows == 0) return FP8Q_OK;
+    if (!x || !q || !sf_mma) return FP8Q_ERR_NULL;
+    if (static_cast<uint64_t>(rows) * k >= (1ull << 31)) return FP8Q_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(sf_mma)) return FP8Q_ERR_ALIGN;
+    DeviceInfo dev;
+    fp8q_status st = current_device(&dev);
+    if (st != FP8Q_OK) return st;
+    return from_cuda(launch_nvfp4_quant(x, q, sf_rowmajor, sf_mma, s2, rows, k, static_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+
+fp8q_status check_nvfp4_gemm_args(const void* qa, const void* sfa, float s2a, const void* qw, const void* sfw,
+                                  float s2w, const void* y, uint32_t m, uint32_t n, uint32_t k) {
+    if (k == 0 || k % 256u || n == 0 || n % kGroup) return FP8Q_ERR_SHAPE;
+    if (!(s2a > 0.0f) || std::isinf(s2a) || !(s2w > 0.0f) || std::isinf(s2w)) return FP8Q_ERR_ARG;
+    if (m == 0) return FP8Q_OK;
+    if (!qa || !sfa || !qw || !sfw || !y) return FP8Q_ERR_NULL;
+    if (static_cast<uint64_t>(m) * k >= (1ull << 31) || static_cast<uint64_t>(n) * k >= (1ull << 31) ||
+        static_cast<uint64_t>(m) * n >= (1ull << 31))
+        return FP8Q_ERR_SHAPE;
+    if (!aligned16(qa) || !aligned16(sfa) || !aligned16(qw) || !aligned16(sfw) || !aligned16(y))
+        return FP8Q_ERR_ALIGN;
+    return FP8Q_OK;
+}
+
+}  // namespace
+
+fp8q_status fp8q_nvfp4_gemm(const void* qa, const void* sfa_mma, float s2a, const void* qw, const void* sfw_mma,
+                            float s2w, void* y, uint32_t m, uint32_t n, uint32_t k, void* stream) {
+    fp8q_status st = check_nvfp4_gemm_args(qa, sfa_mma, s2a, qw, sfw_mma, s2w, y, m, n, k);
+    if (st != FP8Q_OK) return st;
+    if (m == 0) return FP8Q_OK;
+    DeviceInfo dev;
+    if ((st = current_device(&dev)) != FP8Q_OK) return st;
+    Nvfp4GemmLaunch L{qa, sfa_mma, qw, sfw_mma, y, s2a * s2w, m, n, k, false};
+    return from_cuda(launch_nvfp4_gemm(L, static_cast<cudaStream_t>(stream)));
+}
+
+size_t fp8q_nvfp4_linear_workspace_bytes(uint32_t m, uint32_t k) {
+    return round_up(static_cast<size_t>(m) * (k / 2), 256) + round_up(nvfp4_sf_mma_bytes(m, k), 256);
+}
+
+fp8q_status fp8q_nvfp4_linear(const void* x, float s2a, const void* qw, const void* sfw_mma, float s2w, void* y,
+                              void* workspace, size_t workspace_bytes, uint32_t m, uint32_t n, uint32_t k,
+                              void* stream) {
+    if (k == 0 || k % 256u || n == 0 || n % kGroup) return FP8Q_ERR_SHAPE;
+    if (!(s2a > 0.0f) || std::isinf(s2a) || !(s2w > 0.0f) || std::isinf(s2w)) return FP8Q_ERR_ARG;
+    if (m == 0) return FP8Q_OK;
+    if (!x || !qw || !sfw_mma || !y || !workspace) return FP8Q_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FP8Q_ERR_WORKSPACE;
+    if (static_cast<uint64_t>(m) * k >= (1ull << 31)) return FP8Q_ERR_SHAPE;
+    if (workspace_bytes < fp8q_nvfp4_linear_workspace_bytes(m, k)) return FP8Q_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    void* qa = ws;
+    void* sfa = ws + round_up(static_cast<size_t>(m) * (k / 2), 256);
+    fp8q_status st = check_nvfp4_gemm_args(qa, sfa, s2a, qw, sfw_mma, s2w, y, m, n, k);
+    if (st != FP8Q_OK) return st;
+    if (!aligned16(x)) return FP8Q_ERR_ALIGN;
+    DeviceInfo dev;
+    if ((st = current_device(&dev)) != FP8Q_OK) return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = from_cuda(launch_nvfp4_quant(x, qa, nullptr, sfa, s2a, m, k, s))) != FP8Q_OK) return st;
+    // The GEMM is the packer's programmatic dependent: its set-up overlaps
+    // the packer and its producer waits for the packer's grid before loading.
+    Nvfp4GemmLaunch L{qa, sfa, qw, sfw_mma, y, s2a * s2w, m, n, k, true};
+    return from_cuda(launch_nvfp4_gemm(L, s));
+}
+
+fp8q_status fp8q_dequant_fp8_bf16(const void* wq, const float* w_scale, int32_t weight_format, void* y, uint32_t n,
+                                  uint32_t k, void* stream) {
+    if (weight_format != FP8Q_WEIGHT_BLOCK128 && weight_format != FP8Q_WEIGHT_PER_ROW) return FP8Q_ERR_ARG;
+    const bool per_row = weight_format == FP8Q_WEIGHT_PER_ROW;
+    if (k == 0 || k % kGroup || n == 0 || (!per_row && n % kGroup)) return FP8Q_ERR_SHAPE;
+    if (!wq || !w_scale || !y) return FP8Q_ERR_NULL;
+    if (static_cast<uint64_t>(n) * k >= (1ull << 31)) return FP8Q_ERR_SHAPE;
+    if (!aligned16(wq) || !aligned16(w_scale) || !aligned16(y)) return FP8Q_ERR_ALIGN;
+    DeviceInfo dev;
+    fp8q_status st = current_device(&dev);
+    if (st != FP8Q_OK) return st;
+    return from_cuda(launch_dequant_fp8_bf16(wq, w_scale, y, n, k, per_row ? 1u : kGroup, per_row ? k : kGroup,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+fp8q_status fp8q_convert_e2m1(const float* in, uint8_t* out, size_t count, void* stream) {
+    if (!in || !out) return FP8Q_ERR_NULL;
+    if (count == 0) return FP8Q_OK;
+    DeviceInfo dev;
+    fp8q_status st = current_device(&dev);
+    if (st != FP8Q_OK) return st;
+    return from_cuda(launch_convert_e2m1(in, out, count, static_cast<cudaStream_t>(stream)));
+}
+
 fp8q_status fp8q_convert_e4m3(const float* in, uint8_t* out, size_t count, void* stream) {
     if (!in || !out) return FP8Q_ERR_NULL;
     if (count == 0) return FP8Q_OK;
@@ -422,10 +524,13 @@ fp8q_status fp8q_device_error(void* stream, uint32_t* code) {
     DeviceInfo dev;
     fp8q_status st = current_device(&dev);
     if (st != FP8Q_OK) return st;
-    if (read_clear_device_error(code, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    uint32_t nvfp4_code = 0;
+    if (read_clear_device_error(code, static_cast<cudaStream_t>(stream)) != cudaSuccess ||
+        read_clear_nvfp4_error(&nvfp4_code, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
         cudaGetLastError();
         return FP8Q_ERR_CUDA;
     }
+    *code |= nvfp4_code;
     return *code ? FP8Q_ERR_DEVICE_TIMEOUT : FP8Q_OK;
 }
 

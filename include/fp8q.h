@@ -18,7 +18,12 @@
  *     `fp8_act_quant_hopper_reject`), re-derived for the device's SM count;
  *   - the dense FFN that quantizes its input once for the gate and up
  *     projections and quantizes the post-SiLU intermediate once for the down
- *     projection (P-DP, doc of `cublas_fp8_proj_prequant`).
+ *     projection (P-DP, doc of `cublas_fp8_proj_prequant`);
+ *   - the NVFP4 projection arms: E2M1 operands with E4M3 scales per 16
+ *     elements of K on the block-scaled tensor cores, and the FP8-to-bf16
+ *     weight dequantizer the from-FP8 arm starts with (P-DP,
+ *     `cutlass_nvfp4_proj`, `cutlass_nvfp4_proj_from_fp8`,
+ *     `dequant_fp8_bf16_into`).
  *
  * Conventions shared by every call:
  *   - Data pointers are DEVICE pointers owned by the caller, 16-byte aligned.
@@ -27,7 +32,8 @@
  *     only enqueue work; nothing synchronizes.
  *   - bf16 is IEEE bfloat16; e4m3 is OCP FP8 E4M3FN (bias 7, max 448, NaN
  *     only at S.1111.111). Matrices are row-major.
- *   - K and N must be multiples of 128. M == 0 is accepted and launches
+ *   - K and N must be multiples of 128 (the NVFP4 calls state their own K
+ *     rule). M == 0 is accepted and launches
  *     nothing (pointers may then be NULL). M*K, N*K and M*N must stay
  *     below 2^31.
  *   - Every argument is checked before anything is enqueued; a failed check
@@ -330,7 +336,97 @@ fp8q_status fp8q_ffn(const void *x, const void *w_gate_up, const float *w_gate_u
                      void *workspace, size_t workspace_bytes,
                      uint32_t m, uint32_t d, uint32_t i, void *stream);
 
+/* ------------------------------------------------------------ NVFP4 ---- */
+
+/*
+ * NVFP4 projection arms (P-DP, `cutlass_nvfp4_proj`,
+ * `cutlass_nvfp4_weight_transposed_cached`, `cutlass_nvfp4_proj_from_fp8`).
+ * An NVFP4 operand of R rows and K columns is
+ *   q       [R, K/2] bytes of E2M1 codes (1 sign bit, 2 exponent bits with
+ *           bias 1, 1 mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6),
+ *           two to a byte along K, element 2j in the low nibble of byte j.
+ *           This is the [N, K/2] layout the pages' GEMM consumes; their
+ *           [K/2, N] checkpoint layout is its byte transpose.
+ *   scales  one E4M3 code per 16 elements of K, row-major [R, K/16] and in
+ *           the MMA layout the GEMM reads: one 512-byte atom per 128 rows
+ *           (R padded up to a multiple of 128, pad scales zero) and 64
+ *           elements of K, atoms ordered K-fastest within a 128-row block,
+ *           byte (r%32)*16 + ((r%128)/32)*4 + (k/16)%4 inside an atom.
+ *   s2      one fp32 second-level scale (the pages' `weight_scale_2`).
+ * Element (r, k) is worth s2 * e4m3(scale[r][k/16]) * e2m1(q[r][k]).
+ */
+
+/* Bytes of the MMA-layout scales of a rows x k operand: ceil128(rows) * k/16. */
+size_t fp8q_nvfp4_sf_mma_bytes(uint32_t rows, uint32_t k);
+
+/*
+ * Pack bf16 x [rows, k] into NVFP4 with second-level scale s2. Per
+ * 16-element block along K, in fp32:
+ *   sf = e4m3_rne_satfinite(amax / (6 * s2))
+ *   s  = e4m3(sf) * s2
+ *   q  = e2m1_rne_satfinite(x / s)   (IEEE division; a zero s gives zeros
+ *                                     carrying the sign of x)
+ * Writes q [rows, k/2], sf_rowmajor [rows, k/16] (may be NULL) and sf_mma
+ * (fp8q_nvfp4_sf_mma_bytes(rows, k) bytes, pad rows zeroed).
+ * k a multiple of 64; rows*k below 2^31; s2 positive and finite; x, q and
+ * sf_mma 16-byte aligned. rows == 0 returns FP8Q_OK and launches nothing.
+ * Errors: NULL, ALIGN, SHAPE, ARG (s2), UNSUPPORTED_DEVICE, CUDA.
+ */
+fp8q_status fp8q_nvfp4_quant(const void *x, void *q, void *sf_rowmajor, void *sf_mma,
+                             float s2, uint32_t rows, uint32_t k, void *stream);
+
+/*
+ * NVFP4 GEMM on the block-scaled tensor cores:
+ *   y[t][c] = bf16_rn( s2a * s2w * sum_k e2m1(qa[t][k]) * e4m3(sfa[t][k/16])
+ *                                        * e2m1(qw[c][k]) * e4m3(sfw[c][k/16]) )
+ * qa [m, k/2] with its MMA-layout scales sfa_mma, qw [n, k/2] with sfw_mma,
+ * y bf16 [m, n] row-major. k a multiple of 256, n of 128; m*k, n*k and m*n
+ * below 2^31; s2a, s2w positive and finite; every pointer 16-byte aligned.
+ * m == 0 returns FP8Q_OK and launches nothing.
+ * Errors: NULL, ALIGN, SHAPE, ARG, UNSUPPORTED_DEVICE, CUDA.
+ */
+fp8q_status fp8q_nvfp4_gemm(const void *qa, const void *sfa_mma, float s2a,
+                            const void *qw, const void *sfw_mma, float s2w,
+                            void *y, uint32_t m, uint32_t n, uint32_t k, void *stream);
+
+/* Workspace of fp8q_nvfp4_linear: the packed activation at offset 0 (m*k/2
+   bytes, rounded up to 256), then its MMA-layout scales (rounded up to 256). */
+size_t fp8q_nvfp4_linear_workspace_bytes(uint32_t m, uint32_t k);
+
+/*
+ * NVFP4 projection of a bf16 activation x [m, k], packed inside the call as
+ * the pages' projection does: fp8q_nvfp4_quant(x, s2a) into `workspace`
+ * (256-byte aligned, fp8q_nvfp4_linear_workspace_bytes(m, k) bytes), then
+ * fp8q_nvfp4_gemm as its programmatic dependent on `stream`. The pages' call
+ * takes no activation scale: s2a = 1 reproduces it.
+ * Errors: as the two calls, plus WORKSPACE.
+ */
+fp8q_status fp8q_nvfp4_linear(const void *x, float s2a, const void *qw, const void *sfw_mma,
+                              float s2w, void *y, void *workspace, size_t workspace_bytes,
+                              uint32_t m, uint32_t n, uint32_t k, void *stream);
+
+/*
+ * FP8 weight back to bf16 (P-DP, `dequant_fp8_bf16_into`, the first step of
+ * `cutlass_nvfp4_proj_from_fp8`): y[r][c] is the bf16 nearest to the exact
+ * product e4m3(wq[r][c]) * ws(r, c) (ties to even, one rounding), with ws
+ * the weight-format geometry above. k a multiple of 128 (n too for
+ * FP8Q_WEIGHT_BLOCK128); n*k below 2^31; pointers 16-byte aligned.
+ * Packing the result with fp8q_nvfp4_quant(s2 = 1) gives the pages' NVFP4
+ * weight from an FP8 checkpoint.
+ * Errors: NULL, ALIGN, SHAPE, ARG (format), UNSUPPORTED_DEVICE, CUDA.
+ */
+fp8q_status fp8q_dequant_fp8_bf16(const void *wq, const float *w_scale, int32_t weight_format,
+                                  void *y, uint32_t n, uint32_t k, void *stream);
+
 /* ------------------------------------------------------- diagnostics ---- */
+
+/*
+ * Convert `count` fp32 values to E2M1 codes (one per byte, low nibble) with
+ * the conversion fp8q_nvfp4_quant uses (round-to-nearest-even, saturating
+ * at 6). Used to check the conversion exhaustively. Device pointers.
+ * Errors: NULL, UNSUPPORTED_DEVICE, CUDA.
+ */
+fp8q_status fp8q_convert_e2m1(const float *in, uint8_t *out, size_t count, void *stream);
 
 /*
  * Convert `count` fp32 values to e4m3 codes with the same device routine
@@ -372,9 +468,9 @@ fp8q_status fp8q_check_silu_mul(unsigned long long *counts, uint32_t *max_err_bi
 uint64_t fp8q_launch_count(void);
 
 /*
- * Read and clear the device error word of the current device: non-zero when
+ * Read and clear the device error words of the current device: non-zero when
  * a kernel's bounded wait ran out (the kernel then stopped early and its
- * outputs are incomplete). Synchronizes `stream` first. Returns FP8Q_OK or
+ * outputs are incomplete). Bit 0: an FP8 GEMM; bit 1: the NVFP4 GEMM. Synchronizes `stream` first. Returns FP8Q_OK or
  * FP8Q_ERR_DEVICE_TIMEOUT (with *code set), or FP8Q_ERR_CUDA.
  */
 fp8q_status fp8q_device_error(void *stream, uint32_t *code);

@@ -214,6 +214,58 @@ def test_silu_mul_quant_and_ffn_argument_errors():
     assert lib.fp8q_ffn(A, B, C, D, E, A, ws, 1 << 62, 1, d, (1 << 31) + 128, None) == 2
 
 
+def test_nvfp4_argument_errors():
+    lib = _lib.load()
+    # fp8q_nvfp4_quant(x, q, sf_row, sf_mma, s2, rows, k, stream)
+    assert lib.fp8q_nvfp4_quant(A, B, None, C, 1.0, 4, 0, None) == 2
+    assert lib.fp8q_nvfp4_quant(A, B, None, C, 1.0, 4, 32, None) == 2
+    for s2 in (0.0, -1.0, float("inf"), float("nan")):
+        assert lib.fp8q_nvfp4_quant(A, B, None, C, s2, 4, 64, None) == 8
+    assert lib.fp8q_nvfp4_quant(None, None, None, None, 1.0, 0, 64, None) == 0
+    assert lib.fp8q_nvfp4_quant(None, B, None, C, 1.0, 4, 64, None) == 1
+    assert lib.fp8q_nvfp4_quant(A, B, None, None, 1.0, 4, 64, None) == 1
+    assert lib.fp8q_nvfp4_quant(ODD, B, None, C, 1.0, 4, 64, None) == 3
+    assert lib.fp8q_nvfp4_quant(A, B, None, C, 1.0, 1 << 25, 64, None) == 2
+    # fp8q_nvfp4_gemm(qa, sfa, s2a, qw, sfw, s2w, y, m, n, k, stream)
+    assert lib.fp8q_nvfp4_gemm(A, B, 1.0, C, D, 1.0, E, 4, 256, 128, None) == 2    # k % 256
+    assert lib.fp8q_nvfp4_gemm(A, B, 1.0, C, D, 1.0, E, 4, 64, 256, None) == 2     # n % 128
+    assert lib.fp8q_nvfp4_gemm(A, B, 0.0, C, D, 1.0, E, 4, 256, 256, None) == 8
+    assert lib.fp8q_nvfp4_gemm(A, B, 1.0, C, D, float("nan"), E, 4, 256, 256, None) == 8
+    assert lib.fp8q_nvfp4_gemm(None, None, 1.0, None, None, 1.0, None, 0, 256, 256, None) == 0
+    assert lib.fp8q_nvfp4_gemm(A, None, 1.0, C, D, 1.0, E, 4, 256, 256, None) == 1
+    assert lib.fp8q_nvfp4_gemm(A, B, 1.0, C, ODD, 1.0, E, 4, 256, 256, None) == 3
+    assert lib.fp8q_nvfp4_gemm(A, B, 1.0, C, D, 1.0, E, 1 << 23, 256, 256, None) == 2
+    # fp8q_nvfp4_linear(x, s2a, qw, sfw, s2w, y, ws, ws_bytes, m, n, k, stream)
+    m, n, k = 17, 256, 512
+    need = lib.fp8q_nvfp4_linear_workspace_bytes(m, k)
+    ws = ctypes.c_void_p(0x1000000)
+    assert lib.fp8q_nvfp4_linear(A, 1.0, C, D, 1.0, E, ws, need, m, n, 320, None) == 2
+    assert lib.fp8q_nvfp4_linear(A, -2.0, C, D, 1.0, E, ws, need, m, n, k, None) == 8
+    assert lib.fp8q_nvfp4_linear(None, 1.0, None, None, 1.0, None, None, 0, 0, n, k, None) == 0
+    assert lib.fp8q_nvfp4_linear(A, 1.0, C, D, 1.0, None, ws, need, m, n, k, None) == 1
+    assert lib.fp8q_nvfp4_linear(A, 1.0, C, D, 1.0, E, ws, need - 1, m, n, k, None) == 4
+    assert lib.fp8q_nvfp4_linear(A, 1.0, C, D, 1.0, E, ctypes.c_void_p(0x1000010), need, m, n, k, None) == 4
+    assert lib.fp8q_nvfp4_linear(ODD, 1.0, C, D, 1.0, E, ws, need, m, n, k, None) == 3
+    # fp8q_dequant_fp8_bf16(wq, w_scale, format, y, n, k, stream)
+    assert lib.fp8q_dequant_fp8_bf16(A, B, 2, C, 128, 128, None) == 8
+    assert lib.fp8q_dequant_fp8_bf16(A, B, 0, C, 128, 100, None) == 2
+    assert lib.fp8q_dequant_fp8_bf16(A, B, 0, C, 100, 128, None) == 2     # 128 x 128 blocks need n % 128
+    assert lib.fp8q_dequant_fp8_bf16(A, None, 1, C, 100, 128, None) == 1  # per row: any n
+    assert lib.fp8q_dequant_fp8_bf16(A, B, 1, ODD, 100, 128, None) == 3
+    assert lib.fp8q_dequant_fp8_bf16(A, B, 1, C, 1 << 24, 128, None) == 2
+    assert lib.fp8q_convert_e2m1(None, B, 4, None) == 1
+    assert lib.fp8q_convert_e2m1(A, B, 0, None) == 0
+
+
+def test_nvfp4_sizes():
+    lib = _lib.load()
+    for rows, k in [(1, 64), (17, 512), (128, 256), (129, 5120), (1168, 5120), (17408, 5120)]:
+        pad = (rows + 127) // 128 * 128
+        assert lib.fp8q_nvfp4_sf_mma_bytes(rows, k) == pad * k // 16
+        up = lambda v: (v + 255) // 256 * 256
+        assert lib.fp8q_nvfp4_linear_workspace_bytes(rows, k) == up(rows * k // 2) + up(pad * k // 16)
+
+
 def test_ffn_workspace_layout():
     for m, d, i in [(1, 128, 128), (17, 256, 384), (25, 5120, 17408), (1168, 5120, 17408)]:
         off = api.ffn_workspace_layout(m, d, i)
