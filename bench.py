@@ -221,6 +221,25 @@ def weak_scaling_value(units_per_rank_step: float, world: int, steps: int, ms_to
 
 # ------------------------------------------------------------ CPU oracle --
 
+def grow_sample(run, m: int, threads: int, target_s: float):
+    """Rows of a step to time so that `run(rows)` takes about target_s
+    seconds (or all m rows, if they take less). A small first sample carries
+    fixed overheads that make it look slow, so the estimate is refined up to
+    three times. Returns (rows, seconds of the last run)."""
+    threads = max(threads, 1)
+    rows = max(1, min(m, threads))
+    t = run(rows)
+    for _ in range(3):
+        if t >= 0.8 * target_s or rows >= m:
+            break
+        grown = int(min(m, max(rows + 1, rows * target_s / max(t, 1e-3))))
+        if threads <= grown < m:
+            grown -= grown % threads
+        rows = grown
+        t = run(rows)
+    return rows, t
+
+
 def cpu_oracle_sample(wl: dict, seed: int, target_s: float, threads: int, per_row: bool = False):
     """Time the oracle on a bounded sample of one step: quantize R rows of X and
     compute those R rows of the float64 reference output. Returns
@@ -239,11 +258,7 @@ def cpu_oracle_sample(wl: dict, seed: int, target_s: float, threads: int, per_ro
         oracle.gemm_ref(q, s_row, wq, ws, threads=threads)
         return time.perf_counter() - t0
 
-    r = min(m, max(threads, 1))
-    t = run(r)
-    rows = int(min(m, max(r, r * target_s / max(t, 1e-3))))
-    rows = max(threads, rows - rows % max(threads, 1)) if rows >= threads else rows
-    t = run(rows)
+    rows, t = grow_sample(run, m, threads, target_s)
     return 2.0 * rows * n * k / t / 1e12, rows, t
 
 
@@ -498,12 +513,7 @@ def ffn_oracle_sample(wl: dict, threads: int, target_s: float = 10.0):
         oracle.ffn_ref(np.ascontiguousarray(xb[:rows]), wq_gu, ws_gu, wq_dn, ws_dn, threads=threads)
         return time.perf_counter() - t0
 
-    rows = max(1, min(m, threads))
-    t = run(rows)
-    if t < target_s and rows < m:
-        rows = int(min(m, max(rows, rows * target_s / max(t, 1e-3))))
-        rows = max(threads, rows - rows % threads) if rows >= threads else rows
-        t = run(rows)
+    rows, t = grow_sample(run, m, threads, target_s)
     flops = 2.0 * rows * d * 2 * i + 2.0 * rows * i * d
     return flops / t / 1e12, rows, t
 
