@@ -240,7 +240,8 @@ def grow_sample(run, m: int, threads: int, target_s: float):
     return rows, t
 
 
-def cpu_oracle_sample(wl: dict, seed: int, target_s: float, threads: int, per_row: bool = False):
+def cpu_oracle_sample(wl: dict, seed: int, target_s: float, threads: int, per_row: bool = False,
+                      rows: int | None = None):
     """Time the oracle on a bounded sample of one step: quantize R rows of X and
     compute those R rows of the float64 reference output. Returns
     (TFLOP/s equivalent of 2*R*N*K / time, rows, seconds)."""
@@ -258,7 +259,10 @@ def cpu_oracle_sample(wl: dict, seed: int, target_s: float, threads: int, per_ro
         oracle.gemm_ref(q, s_row, wq, ws, threads=threads)
         return time.perf_counter() - t0
 
-    rows, t = grow_sample(run, m, threads, target_s)
+    if rows is None:
+        rows, t = grow_sample(run, m, threads, target_s)
+    else:
+        t = run(rows)
     return 2.0 * rows * n * k / t / 1e12, rows, t
 
 
@@ -271,9 +275,9 @@ def reference_arm(args):
     threads = os.cpu_count() or 1
     per_step = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
     vals = []
-    rows = 0
+    rows = None  # sized in the first warm-up step, then the same sample every step
     for i in range(args.warmup + args.steps):
-        v, rows, _ = cpu_oracle_sample(wl, 1000 + wl["number"], per_step, threads)
+        v, rows, _ = cpu_oracle_sample(wl, 1000 + wl["number"], per_step, threads, rows=rows)
         if i >= args.warmup:
             vals.append(v)
     value = statistics.median(vals)
@@ -494,7 +498,7 @@ def ours_arm(args):
 _FFN_ORACLE_W = {}
 
 
-def ffn_oracle_sample(wl: dict, threads: int, target_s: float = 10.0):
+def ffn_oracle_sample(wl: dict, threads: int, target_s: float = 10.0, rows: int | None = None):
     """Time the oracle's FFN on a bounded sample of one step's token rows;
     returns (TFLOP/s equivalent, rows, seconds). Weight preparation is not
     part of the step and is done once."""
@@ -513,7 +517,10 @@ def ffn_oracle_sample(wl: dict, threads: int, target_s: float = 10.0):
         oracle.ffn_ref(np.ascontiguousarray(xb[:rows]), wq_gu, ws_gu, wq_dn, ws_dn, threads=threads)
         return time.perf_counter() - t0
 
-    rows, t = grow_sample(run, m, threads, target_s)
+    if rows is None:
+        rows, t = grow_sample(run, m, threads, target_s)
+    else:
+        t = run(rows)
     flops = 2.0 * rows * d * 2 * i + 2.0 * rows * i * d
     return flops / t / 1e12, rows, t
 
@@ -524,9 +531,10 @@ def ffn_reference_arm(args):
     wl = FFN_WORKLOADS[args.workload]
     threads = os.cpu_count() or 1
     vals = []
-    rows = 0
+    rows = None  # sized in the first warm-up step, then the same sample every step
+    per_step = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
     for j in range(args.warmup + args.steps):
-        v, rows, _ = ffn_oracle_sample(wl, threads, target_s=max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup))))
+        v, rows, _ = ffn_oracle_sample(wl, threads, target_s=per_step, rows=rows)
         if j >= args.warmup:
             vals.append(v)
     value = statistics.median(vals)
