@@ -5,6 +5,8 @@ way: a library decoder (torch's float8_e4m3fn), closed forms worked by hand,
 an error bound, brute force with an independent decoder, exact integer
 arithmetic, and a negative control with the wrong scale layout.
 """
+from fractions import Fraction
+
 import numpy as np
 import pytest
 import torch
@@ -197,6 +199,71 @@ def test_bf16_subnormal_inputs(oracle_mod):
     assert np.all(q[0, 0::2] == 0x00) and np.all(q[0, 1::2] == 0x80)
 
 
+# ------------------------------------------ division, not reciprocal --
+
+def _rn24(v: Fraction) -> Fraction:
+    """The binary32 value nearest to a positive normal-range rational, ties to
+    even, by exact integer arithmetic."""
+    e = v.numerator.bit_length() - v.denominator.bit_length()
+    if Fraction(2) ** e > v:
+        e -= 1
+    if Fraction(2) ** (e + 1) <= v:
+        e += 1
+    quantum = Fraction(2) ** (e - 23)
+    return round(v / quantum) * quantum  # Fraction.__round__ rounds half to even
+
+
+def _e4m3_nearest(t: Fraction) -> int:
+    """Nearest finite E4M3 code to a rational (OCP E4M3FN grid, ties to the
+    even mantissa, saturating at 448), by exhaustive comparison."""
+    sign = 0x80 if t < 0 else 0
+    a = abs(t)
+    best = None
+    for c in range(0x7F):
+        e, m = c >> 3, c & 7
+        v = Fraction(m, 8) * Fraction(1, 64) if e == 0 else (1 + Fraction(m, 8)) * Fraction(2) ** (e - 7)
+        key = (abs(v - a), c & 1)
+        if best is None or key < best[0]:
+            best = (key, c)
+    return sign | best[1]
+
+
+def _bf16_value(bits: int) -> Fraction:
+    return Fraction(float(np.array([bits << 16], np.uint32).view(np.float32)[0]))
+
+
+def test_codes_follow_ieee_division_not_a_reciprocal_product(oracle_mod):
+    """The quotient x / s is one IEEE fp32 division. Multiplying by the
+    rounded reciprocal instead changes some codes; such (x, amax) pairs are
+    searched for, and each code is decided with exact rational arithmetic."""
+    rng = np.random.default_rng(0)
+    xs_bits = np.arange(0, 0x7F80, dtype=np.uint32)
+    xs = (xs_bits << 16).view(np.float32)
+    witnesses = []
+    for ab in rng.integers(0x3C00, 0x4700, 400):
+        amax = np.float32((np.uint32(ab) << np.uint32(16)).view(np.float32))
+        s = amax / np.float32(448.0)
+        xv = xs[xs <= amax]
+        by_div = torch_encode(xv / s)
+        by_rcp = torch_encode(xv * (np.float32(1.0) / s))
+        for i in np.nonzero(by_div != by_rcp)[0][:2]:
+            witnesses.append((int(ab), int(xv[i].view(np.uint32) >> 16)))
+        if len(witnesses) >= 6:
+            break
+    assert len(witnesses) >= 6
+    for amax_bits, x_bits in witnesses:
+        amax, x = _bf16_value(amax_bits), _bf16_value(x_bits)
+        s = _rn24(amax / 448)
+        want = _e4m3_nearest(_rn24(x / s))
+        other = _e4m3_nearest(_rn24(x * _rn24(1 / s)))
+        assert want != other
+        row = np.zeros((1, 128), np.uint16)
+        row[0, 0], row[0, 1] = amax_bits, x_bits
+        q, s_r, _ = oracle_mod.quant_act(row)
+        assert Fraction(float(s_r[0, 0])) == s
+        assert q[0, 1] == want, (hex(amax_bits), hex(x_bits))
+
+
 # ------------------------------------------------------- error bounds --
 
 def _check_quant_error_bound(x_f32, q, scale_of):
@@ -322,6 +389,19 @@ def test_tolerance_accepts_bf16_rounding_and_rejects_wrong_layout(oracle_mod):
     assert rel_rms > 1e-2
     # a 2 % gain error is also rejected
     assert oracle_mod.check_tolerance(inputs.f32_to_bf16_bits((ref * 1.02).astype(np.float32)), ref)[0] > 0
+
+
+def test_tolerance_formula_by_hand(oracle_mod):
+    """|y - ref| <= 8e-3 |ref| + 1e-3 rms(ref), rms over every compared
+    element. ref = [100, 0, 0, 0]: rms = 50, so the bounds are 0.85 and 0.05."""
+    ref = np.array([100.0, 0.0, 0.0, 0.0])
+    y = inputs.f32_to_bf16_bits(np.array([100.5, 0.046875, -0.046875, 0.0625], np.float32))
+    bad, worst = oracle_mod.check_tolerance(y, ref)
+    assert bad == 1 and worst == pytest.approx(0.0625 / 0.05)
+    # mostly the relative term: ref [1000, 0] (rms 707.1, bound 8 + 0.71 = 8.71)
+    ref = np.array([1000.0, 0.0])
+    assert oracle_mod.check_tolerance(inputs.f32_to_bf16_bits(np.array([1008.0, 0.0], np.float32)), ref)[0] == 0
+    assert oracle_mod.check_tolerance(inputs.f32_to_bf16_bits(np.array([1016.0, 0.0], np.float32)), ref)[0] == 1
 
 
 def test_inputs_are_deterministic_and_shaped():
