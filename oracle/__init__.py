@@ -267,6 +267,24 @@ def silu_mul_quant(gate_bf16: np.ndarray, up_bf16: np.ndarray):
     return q, s_row, s_k
 
 
+def silu_mul_quant_stacked(gate_up_bf16: np.ndarray):
+    """silu_mul_quant over the two halves of one [M, 2I] array (gate columns
+    first), read in place with row stride 2I."""
+    gu = np.ascontiguousarray(gate_up_bf16, dtype=np.uint16)
+    m, two_i = gu.shape
+    i = two_i // 2
+    if i % GROUP or two_i != 2 * i:
+        raise ValueError("the intermediate width must be a multiple of 128")
+    q = np.empty((m, i), np.uint8)
+    s_row = np.empty((m, i // GROUP), np.float32)
+    s_k = np.empty((i // GROUP, m_pad(m)), np.float32)
+    lib = _load()
+    up = ctypes.c_void_p(gu.ctypes.data + 2 * i)  # bytes to the first up column
+    rc = lib.oracle_silu_mul_quant(_ptr(gu), up, two_i, m, i, _ptr(q), _ptr(s_row), _ptr(s_k))
+    assert rc == 0
+    return q, s_row, s_k
+
+
 def ffn_ref(x_bf16: np.ndarray, wq_gate_up: np.ndarray, ws_gate_up: np.ndarray,
             wq_down: np.ndarray, ws_down: np.ndarray, threads: int = 1) -> dict:
     """The dense FFN, each stage by its definition:

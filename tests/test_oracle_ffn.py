@@ -202,6 +202,18 @@ def test_silu_mul_quant_is_quant_of_h(oracle_mod, m):
     assert s_k.shape == (i // 128, mp) and not np.any(s_k[:, m:].view(np.uint32))
 
 
+def test_silu_mul_quant_reads_stacked_halves_in_place(oracle_mod):
+    # gate and up as the two halves of one [m, 2i] row (row stride 2i): the
+    # same result as contiguous copies of the halves
+    m, i = 5, 256
+    rng = np.random.default_rng(9)
+    gu = bf16(rng.normal(0, 3, (m, 2 * i)))
+    got = oracle_mod.silu_mul_quant_stacked(gu)
+    want = oracle_mod.silu_mul_quant(np.ascontiguousarray(gu[:, :i]), np.ascontiguousarray(gu[:, i:]))
+    for a, b in zip(got, want):
+        assert np.array_equal(a.view(np.uint8), b.view(np.uint8))
+
+
 # ------------------------------------------------------- FFN composition --
 
 def deq(codes):
