@@ -45,6 +45,19 @@ def test_library_exports_every_declared_symbol():
     assert set(_lib.SIGNATURES) == set(names)
 
 
+def test_c_program_uses_the_abi(tmp_path):
+    """include/fp8q.h compiles as pedantic C99, and a C program linked against
+    libfp8q.so gets the same answers as the ctypes binding (tests/c_abi_host.c)."""
+    lib_dir = os.path.dirname(_lib.LIB_PATH)
+    exe = str(tmp_path / "c_abi_host")
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                           "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c_abi_host.c"),
+                           "-L", lib_dir, "-lfp8q", f"-Wl,-rpath,{lib_dir}", "-o", exe])
+    out = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.strip() == "ok"
+
+
 def test_status_strings_and_version():
     lib = _lib.load()
     for code in range(0, 9):
