@@ -299,3 +299,26 @@ def test_no_device_reports_cuda_error_not_crash():
     assert lib.fp8q_quant_act(A, B, C, D, 16, 512, None) in (5, 7)
     code = ctypes.c_uint32(0)
     assert lib.fp8q_device_error(None, ctypes.byref(code)) in (5, 7)
+
+
+def test_cpu_baseline_sample_sizing():
+    """bench.grow_sample: the CPU oracle baseline times about target seconds
+    of work (or the whole step), refining a small first probe's estimate."""
+    import bench
+
+    calls = []
+
+    def fake(per_row, fixed=0.3):
+        def run(rows):
+            calls.append(rows)
+            return fixed + rows * per_row
+        return run
+
+    rows, t = bench.grow_sample(fake(0.01), 1168, 16, 10.0)
+    assert calls[0] == 16 and rows % 16 == 0 and 8.0 <= t and len(calls) <= 4
+    calls.clear()
+    rows, t = bench.grow_sample(fake(0.01), 100, 16, 10.0)     # the whole step takes less than the target
+    assert rows == 100 and calls == [16, 100]
+    calls.clear()
+    rows, t = bench.grow_sample(fake(1.0), 1168, 16, 10.0)      # the probe alone exceeds the target
+    assert rows == 16 and calls == [16]
