@@ -465,9 +465,13 @@ def ours_arm(args):
         threads = os.cpu_count() or 1
         v, rows, t = cpu_oracle_sample(wl, seed_base, args.cpu_seconds, threads,
                                        per_row=args.weight_format == "per_row")
+        v1, rows1, t1 = cpu_oracle_sample(wl, seed_base, args.cpu_seconds / 2, 1,
+                                          per_row=args.weight_format == "per_row")
         cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": f"{rows} of {m} token rows of one step (quantize + float64 GEMM rows), "
-                         f"{t:.1f} s, scaled to TFLOP/s"}
+                         f"{t:.1f} s, scaled to TFLOP/s",
+               "single_thread": {"value": v1, "unit": "TFLOP/s", "cores": 1,
+                                 "sample": f"{rows1} of {m} token rows, {t1:.1f} s"}}
 
     if rank == 0:
         line = {
@@ -655,8 +659,11 @@ def ffn_arm(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = os.cpu_count() or 1
         v, rows, t = ffn_oracle_sample(wl, threads, target_s=args.cpu_seconds)
+        v1, rows1, t1 = ffn_oracle_sample(wl, 1, target_s=args.cpu_seconds / 2)
         cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": f"{rows} of {m} token rows of one FFN step, {t:.1f} s, scaled to TFLOP/s"}
+               "sample": f"{rows} of {m} token rows of one FFN step, {t:.1f} s, scaled to TFLOP/s",
+               "single_thread": {"value": v1, "unit": "TFLOP/s", "cores": 1,
+                                 "sample": f"{rows1} of {m} token rows, {t1:.1f} s"}}
     if rank == 0:
         line = {
             "metric": FFN_METRIC, "value": weak_scaling_value(flops, world, 1, ms) / 1e12, "unit": "TFLOP/s",
