@@ -9,6 +9,9 @@ if ROOT not in sys.path:
 
 
 def pytest_configure(config):
+    # GPU tests are selected with -m gpu / -m "not gpu". Without a device
+    # they fail instead of skipping, so a machine whose GPU cannot be used
+    # never reports a green GPU run.
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
 
 
