@@ -271,6 +271,20 @@ def cpu_oracle_sample(wl: dict, seed: int, target_s: float, threads: int, per_ro
     return 2.0 * rows * n * k / t / 1e12, rows, t
 
 
+def cpu_oracle_quant(wl: dict, seed: int):
+    """The oracle's activation quantizer over the step's whole [M, K]
+    activation, single-threaded: (GB/s with the GPU kernel's byte count,
+    seconds)."""
+    import oracle
+    from fp8_block_scaled_group_b200 import inputs
+    m, k = wl["m"], wl["k"]
+    xb = inputs.activations(m, k, seed, wl["p"], wl["sigma"])
+    t0 = time.perf_counter()
+    oracle.quant_act(xb)
+    t = time.perf_counter() - t0
+    return quant_bytes(m, k) / t / 1e9, t
+
+
 def reference_arm(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -478,6 +492,9 @@ def ours_arm(args):
                          f"{t:.1f} s, scaled to TFLOP/s",
                "single_thread": {"value": v1, "unit": "TFLOP/s", "cores": 1,
                                  "sample": f"{rows1} of {m} token rows, {t1:.1f} s"}}
+        qv, qt = cpu_oracle_quant(wl, seed_base)
+        cpu["quantizer"] = {"value": qv, "unit": "GB/s", "cores": 1,
+                            "sample": f"the whole [{m}, {k}] activation, {qt:.2f} s"}
 
     if rank == 0:
         line = {
