@@ -62,10 +62,13 @@ def load_peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def quant_bytes(m, k):
+def quant_bytes(m, k, row_major=True):
+    """Algorithmic HBM bytes of one fp8q_quant_act call: read X (2 B an
+    element), write Q (1 B), the K-major scales with their pad rows and, as
+    the call emits them, the row-major scales (4 B a group each)."""
     g = k // 128
     mp = -(-m // 16) * 16
-    return 2 * m * k + m * k + 4 * g * mp  # read X, write Q and the K-major scales
+    return 2 * m * k + m * k + 4 * g * mp + (4 * g * m if row_major else 0)
 
 
 def gemm_hbm_bytes(m, n, k):
@@ -224,6 +227,197 @@ def weak_scaling_value(units_per_rank_step: float, world: int, steps: int, ms_to
     return units_per_rank_step * world * steps / (ms_total * 1e-3)
 
 
+def hold_stream(steps: int):
+    """A spin kernel ahead of timed launches keeps the GPU busy while the host
+    enqueues them, so the device runs them back to back and the events
+    measure device time, not host launch overhead."""
+    import torch
+    torch.cuda._sleep(int(2e6 + 2e5 * steps))
+
+
+def stream_loop_ms(fn, steps: int) -> float:
+    """Average device time per call of `steps` calls launched back to back on
+    the current stream (CUDA events on that stream)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    hold_stream(steps)
+    e0.record(stream)
+    for i in range(steps):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def graph_loop_ms(fn, steps: int, replays: int = 5) -> float:
+    """Average device time per call of `steps` calls captured in one CUDA
+    graph (no host launch work between them), median over `replays` replays,
+    CUDA events on the replaying stream. `fn` must have run before (set-up
+    such as shared-memory opt-in happens on first calls, outside capture)."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            for i in range(steps):
+                fn(i)
+    torch.cuda.synchronize()
+    graph.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    times = []
+    for _ in range(replays):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / steps)
+    del graph
+    return statistics.median(times)
+
+
+L2_BYTES = 126 * 2 ** 20
+
+
+def rotation(bytes_per_set: int, lo: int = 2, hi: int = 24) -> int:
+    """Input sets to rotate so that one pass over them moves more than 3x the
+    L2 size: no launch reads what an earlier one left in L2."""
+    return max(lo, min(hi, -(-3 * L2_BYTES // max(1, bytes_per_set))))
+
+
+def device_activations(m: int, k: int, p: float, sigma: float, gen, dev):
+    """Seeded synthetic activations drawn on the device, for timing only: bf16
+    N(0,1) with a fraction p of entries replaced by N(0, sigma) outliers."""
+    import torch
+    x = torch.randn((m, k), generator=gen, device=dev, dtype=torch.float32)
+    mask = torch.rand((m, k), generator=gen, device=dev) < p
+    x = torch.where(mask, torch.randn((m, k), generator=gen, device=dev) * sigma, x)
+    return x.to(torch.bfloat16)
+
+
+def kernel_timings(wl: dict, dev, sms: int, hbm: float, fp8_peak: float, steps: int, warmup: int,
+                   decode_variants: bool = True) -> dict:
+    """Isolated device timings of one workload's kernels, each in its own loop
+    over rotating inputs larger than L2: the GEMM, the activation quantizer
+    (with both scale layouts, as fp8q_quant_act emits them) and the fused
+    linear. Each loop is timed twice, launched back to back on the stream and
+    captured in a CUDA graph; fractions use the graph figure (no host launch
+    work between kernels), the stream figure is reported beside it."""
+    import torch
+    from fp8_block_scaled_group_b200 import api
+    m, n, k = wl["m"], wl["n"], wl["k"]
+    g, mp = k // 128, api.m_pad(m)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7000 + wl["number"] * 131 + m)
+    reps = max(steps, 20)
+
+    def both(fn, nsets):
+        for i in range(max(warmup, nsets)):
+            fn(i)
+        torch.cuda.synchronize()
+        st = stream_loop_ms(fn, max(reps, 2 * nsets))
+        gr = graph_loop_ms(fn, max(reps, 2 * nsets))
+        return st * 1e3, gr * 1e3
+
+    out = {"m": m, "n": n, "k": k}
+    # activation quantizer
+    qb = quant_bytes(m, k)
+    nq = rotation(qb)
+    xs = [device_activations(m, k, wl["p"], wl["sigma"], gen, dev) for _ in range(min(nq, 3))]
+    xs += [xs[i % len(xs)].clone() for i in range(len(xs), nq)]
+    qo = [(torch.empty((m, k), dtype=torch.uint8, device=dev), torch.empty((m, g), dtype=torch.float32, device=dev),
+           torch.empty((g, mp), dtype=torch.float32, device=dev)) for _ in range(nq)]
+    pick = api.quant_pick(m, k, sms)
+    picked = "multi" if pick.variant == api.MULTI else "single"
+    variants = ["single", "multi"] if (decode_variants and m <= 64) else [picked]
+    aq = {"bound": "hbm", "bytes": qb, "picked": picked, "peak": hbm, "unit": "GB/s"}
+    for name in variants:
+        var = api.MULTI if name == "multi" else api.SINGLE
+        st, gr = both(lambda i, var=var: api.quant_act(xs[i % nq], variant=var, out=qo[i % nq]), nq)
+        aq[name] = {"us_graph": gr, "us_stream": st}
+    aq["us"] = aq[picked]["us_graph"]
+    aq["us_stream"] = aq[picked]["us_stream"]
+    aq["achieved"] = qb / (aq["us"] * 1e-6) / 1e9
+    aq["frac"] = aq["achieved"] / hbm
+    aq["frac_stream"] = qb / (aq["us_stream"] * 1e-6) / 1e9 / hbm
+    out["act_quant"] = aq
+    del xs, qo
+    torch.cuda.empty_cache()
+    # GEMM and fused linear over rotating weights
+    gb = gemm_hbm_bytes(m, n, k)
+    ns = rotation(n * k + m * k * 3 + 2 * m * n)
+    x0 = device_activations(m, k, wl["p"], wl["sigma"], gen, dev)
+    q0, _, s0 = api.quant_act(x0)
+    sets = []
+    for i in range(ns):
+        w = (torch.randn((n, k), generator=gen, device=dev, dtype=torch.float32) * 0.02).to(torch.bfloat16)
+        wq, ws = api.quant_weight(w)
+        del w
+        sets.append(dict(x=x0 if i == 0 else x0.clone(), q=q0 if i == 0 else q0.clone(),
+                         s=s0 if i == 0 else s0.clone(), wq=wq, ws=ws,
+                         work=torch.empty(api.linear_workspace_bytes(m, k), dtype=torch.uint8, device=dev),
+                         y=torch.empty((m, n), dtype=torch.bfloat16, device=dev)))
+    st, gr = both(lambda i: api.gemm_blockscaled(sets[i % ns]["q"], sets[i % ns]["s"], sets[i % ns]["wq"],
+                                                 sets[i % ns]["ws"], out=sets[i % ns]["y"]), ns)
+    flops = 2.0 * m * n * k
+    if m <= 64:
+        gm = {"bound": "hbm", "kernel": "gemm_decode_kernel", "unit": "GB/s", "peak": hbm,
+              "achieved": gb / (gr * 1e-6) / 1e9, "frac_stream": gb / (st * 1e-6) / 1e9 / hbm}
+    else:
+        gm = {"bound": "tensor", "kernel": "gemm_blockscaled_kernel", "unit": "TFLOP/s", "peak": fp8_peak,
+              "achieved": flops / (gr * 1e-6) / 1e12, "frac_stream": flops / (st * 1e-6) / 1e12 / fp8_peak}
+    gm["frac"] = gm["achieved"] / gm["peak"]
+    gm.update(us_graph=gr, us_stream=st, algorithmic_bytes=gb, tflops=flops / (gr * 1e-6) / 1e12)
+    out["gemm"] = gm
+    st, gr = both(lambda i: api.linear(sets[i % ns]["x"], sets[i % ns]["wq"], sets[i % ns]["ws"],
+                                       workspace=sets[i % ns]["work"], out=sets[i % ns]["y"]), ns)
+    out["linear"] = {"us_graph": gr, "us_stream": st, "tflops_graph": flops / (gr * 1e-6) / 1e12}
+    out["rotation"] = {"quantizer_sets": nq, "gemm_sets": ns}
+    del sets
+    torch.cuda.empty_cache()
+    return out
+
+
+def decode_quant_arms(dev, sms: int, warmup: int) -> list:
+    """Both activation-quantizer variants at every decode-width arm of the
+    pages' table (M in 16, 17, 25 and K in 5120, 6144, 17408), each in a CUDA
+    graph over rotating inputs: the picked variant must not be the slower."""
+    import torch
+    from fp8_block_scaled_group_b200 import api
+    rows = []
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7777)
+    for k in (5120, 6144, 17408):
+        for m in (16, 17, 25):
+            g, mp = k // 128, api.m_pad(m)
+            nq = 16
+            xs = [device_activations(m, k, 0.01, 20.0, gen, dev) for _ in range(nq)]
+            qo = [(torch.empty((m, k), dtype=torch.uint8, device=dev), torch.empty((m, g), dtype=torch.float32, device=dev),
+                   torch.empty((g, mp), dtype=torch.float32, device=dev)) for _ in range(nq)]
+            row = {"m": m, "k": k}
+            for name, var in (("single", api.SINGLE), ("multi", api.MULTI)):
+                fn = lambda i, var=var: api.quant_act(xs[i % nq], variant=var, out=qo[i % nq])
+                for i in range(max(warmup, nq)):
+                    fn(i)
+                torch.cuda.synchronize()
+                row[name + "_us"] = graph_loop_ms(fn, 64) * 1e3
+            row["picked"] = "multi" if api.quant_pick(m, k, sms).variant == api.MULTI else "single"
+            row["faster"] = "multi" if row["multi_us"] < row["single_us"] else "single"
+            rows.append(row)
+    return rows
+
+
+# The configurations besides the headline one, timed kernel by kernel:
+# decode widths at both K and the M=4576 prefill at both K.
+PER_CONFIG = ["decode_m25_n6144_k5120", "decode_m25_n5120_k17408",
+              "prefill_m4576_n6144_k6144", "prefill_m4576_n6144_k17408"]
+
+
 # ------------------------------------------------------------ CPU oracle --
 
 def grow_sample(run, m: int, threads: int, target_s: float):
@@ -304,6 +498,8 @@ def reference_arm(args):
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": flops / (value * 1e12) * 1e3,
+        "ms_per_step_kind": f"extrapolated: each step times {rows} of {wl['m']} token rows and scales that "
+                            f"time to the whole step",
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "m": wl["m"], "n": wl["n"], "k": wl["k"]},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
@@ -341,6 +537,13 @@ def ours_arm(args):
         work = torch.empty(api.linear_workspace_bytes(m, k), dtype=torch.uint8, device=dev)
         y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
         sets.append(dict(x=x, wq=wq, ws=ws, work=work, y=y, xb=xb))
+    # More sets (copies in distinct memory) until a pass over them moves more
+    # than 3x L2, so that no step reads what an earlier step left in L2.
+    n_sets = rotation(m * k * 3 + n * k + 2 * m * n, lo=N_SETS)
+    for i in range(N_SETS, n_sets):
+        b = sets[i % N_SETS]
+        sets.append(dict(x=b["x"].clone(), wq=b["wq"].clone(), ws=b["ws"].clone(), work=torch.empty_like(b["work"]),
+                         y=torch.empty_like(b["y"]), xb=b["xb"]))
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
@@ -349,19 +552,13 @@ def ours_arm(args):
         raise SystemExit("--decode-path fused serves at most 32 tokens")
 
     def step(i):
-        s = sets[i % N_SETS]
+        s = sets[i % n_sets]
         linear_call(s["x"], s["wq"], s["ws"], workspace=s["work"], out=s["y"])
 
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
     barrier(world)
-
-    def hold_stream(steps: int):
-        # A spin kernel ahead of the timed launches keeps the GPU busy while
-        # the host enqueues them, so the device runs them back to back and
-        # the events measure device time, not host launch overhead.
-        torch.cuda._sleep(int(2e6 + 2e5 * steps))
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -381,60 +578,30 @@ def ours_arm(args):
     launches = api.launch_count() - launches0
     ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
 
-    # Per-kernel timing, each kernel alone in its own back-to-back loop on the
-    # launching stream. The GEMM rotates the three full input sets; the
-    # quantizer rotates its own inputs and outputs over more than 3x L2, so
-    # neither reads what the previous launch left in L2 and neither pays for
-    # the other's deferred write-backs.
-    off = api.linear_scale_offset(m, k)
-    mp = api.m_pad(m)
-
-    def q_views(work):
-        return work[:m * k].view(m, k), work[off:off + 4 * g * mp].view(torch.float32).view(g, mp)
-
-    views = [q_views(s["work"]) for s in sets]
-    for i in range(N_SETS):  # the GEMM's inputs: each set's own quantized X
-        api.quant_act(sets[i]["x"], out=(views[i][0], None, views[i][1]))
-    n_q = max(N_SETS, min(64, -(-3 * 126 * 2 ** 20 // (3 * m * k))))
-    qx = [sets[i % N_SETS]["x"] if i < N_SETS else sets[i % N_SETS]["x"].clone() for i in range(n_q)]
-    qw = [torch.empty_like(sets[0]["work"]) for _ in range(n_q)]
-    qv = [q_views(w) for w in qw]
-    for i in range(n_q):
-        api.quant_act(qx[i], out=(qv[i][0], None, qv[i][1]))
-    torch.cuda.synchronize()
-
-    def time_loop(fn, steps):
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        hold_stream(steps)
-        e0.record(stream)
-        for i in range(steps):
-            fn(i)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / steps
-
-    def gemm_only(i):
-        s = sets[i % N_SETS]
-        api.gemm_blockscaled(views[i % N_SETS][0], views[i % N_SETS][1], s["wq"], s["ws"], out=s["y"])
-
-    def quant_only(i):
-        api.quant_act(qx[i % n_q], out=(qv[i % n_q][0], None, qv[i % n_q][1]))
-
-    q_steps = max(args.steps, 2 * n_q)
-    g_ms = [time_loop(gemm_only, args.steps)]
-    q_ms = [time_loop(quant_only, q_steps)]
-    del qx, qw, qv
+    # Per-kernel timing, each kernel alone in its own loop over rotating
+    # inputs larger than L2 (kernel_timings): the headline workload, then the
+    # other configurations, and the decode-width arms of the quantizer's two
+    # variants. The clocks keep being sampled throughout.
+    hbm, bf16, bf16_sus, src = load_peaks()
+    fp8_peak = bf16 * 2.0  # fp8 dense = 2x bf16 dense (nominal 4.5 / 2.25 PF)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    kt = kernel_timings(wl, dev, sms, hbm, fp8_peak, args.steps, args.warmup)
+    per_config = {}
+    if not args.no_per_config:
+        for name in PER_CONFIG:
+            if name != args.workload:
+                per_config[name] = kernel_timings(WORKLOADS[name], dev, sms, hbm, fp8_peak, args.steps, args.warmup)
+        per_config["act_quant_decode_arms"] = decode_quant_arms(dev, sms, args.warmup)
     clk = clocks.stop()
 
     # End to end through the public call with host buffers: pinned X in,
     # fused linear, Y back to pinned host memory, every step.
-    x_host = [torch.from_numpy(s["xb"].view(np.int16)).view(torch.bfloat16).pin_memory() for s in sets]
+    x_host = [torch.from_numpy(s["xb"].view(np.int16)).view(torch.bfloat16).pin_memory() for s in sets[:N_SETS]]
     y_host = torch.empty((m, n), dtype=torch.bfloat16).pin_memory()
     x_dev = torch.empty((m, k), dtype=torch.bfloat16, device=dev)
 
     def e2e_step(i):
-        s = sets[i % N_SETS]
+        s = sets[i % n_sets]
         x_dev.copy_(x_host[i % N_SETS], non_blocking=True)
         linear_call(x_dev, s["wq"], s["ws"], workspace=s["work"], out=s["y"])
         y_host.copy_(s["y"], non_blocking=True)
@@ -455,30 +622,30 @@ def ours_arm(args):
     flops = 2.0 * m * n * k
     value = weak_scaling_value(flops, world, args.steps, ms_total) / 1e12
     e2e_value = weak_scaling_value(flops, world, args.steps, e2e_ms) / 1e12
-    hbm, bf16, bf16_sus, src = load_peaks()
-    fp8_peak = bf16 * 2.0  # fp8 dense = 2x bf16 dense (nominal 4.5 / 2.25 PF)
-    gemm_us = statistics.mean(g_ms) * 1e3
-    quant_us = statistics.mean(q_ms) * 1e3
-    gemm_tf = flops / (gemm_us * 1e-6) / 1e12
-    quant_gbs = quant_bytes(m, k) / (quant_us * 1e-6) / 1e9
-    q_kernel = "quant_act_multi_kernel" if api.quant_pick(m, k, torch.cuda.get_device_properties(dev).multi_processor_count).variant == api.MULTI else "quant_act_single_kernel"
+    q_kernel = "quant_act_stream_kernel" if kt["act_quant"]["picked"] == "multi" else "quant_act_single_kernel"
     q_traffic = read_traffic(q_kernel, args.workload)
-    if m <= 64:
-        # Decode widths stream the weight: the GEMM is bound by HBM bytes.
-        g_kernel = "gemm_decode_kernel"
-        g_bytes = gemm_hbm_bytes(m, n, k)
-        g_gbs = g_bytes / (gemm_us * 1e-6) / 1e9
-        roofline = {"bound": "hbm", "kernel": g_kernel, "achieved": g_gbs, "peak": hbm, "unit": "GB/s",
-                    "frac": g_gbs / hbm, "traffic": read_traffic(g_kernel, args.workload),
-                    "peak_source": f"{src} copy bandwidth", "algorithmic_bytes": g_bytes, "us": gemm_us,
-                    "tflops": gemm_tf}
+    gm = kt["gemm"]
+    g_kernel = gm["kernel"]
+    roofline = {"bound": gm["bound"], "kernel": g_kernel, "achieved": gm["achieved"], "peak": gm["peak"],
+                "unit": gm["unit"], "frac": gm["frac"], "traffic": read_traffic(g_kernel, args.workload),
+                "algorithmic_bytes": gm["algorithmic_bytes"], "us": gm["us_graph"], "us_stream_loop": gm["us_stream"],
+                "frac_stream_loop": gm["frac_stream"], "tflops": gm["tflops"],
+                "timing": "CUDA events around a CUDA graph of back-to-back launches over rotating inputs > L2; "
+                          "us_stream_loop: the same launches enqueued on the stream"}
+    if gm["bound"] == "hbm":
+        roofline["peak_source"] = f"{src} copy bandwidth"
     else:
-        g_kernel = "gemm_blockscaled_kernel"
-        roofline = {"bound": "tensor", "kernel": g_kernel, "achieved": gemm_tf, "peak": fp8_peak, "unit": "TFLOP/s",
-                    "frac": gemm_tf / fp8_peak, "traffic": read_traffic(g_kernel, args.workload),
-                    "peak_source": f"{src} bf16 burst x 2 (fp8:bf16 nominal ratio)",
-                    "frac_of_nominal_fp8": gemm_tf / FP8_NOMINAL_TFLOPS,
-                    "algorithmic_bytes": gemm_hbm_bytes(m, n, k), "us": gemm_us}
+        roofline["peak_source"] = f"{src} bf16 burst x 2 (fp8:bf16 nominal ratio)"
+        roofline["frac_of_nominal_fp8"] = gm["achieved"] / FP8_NOMINAL_TFLOPS
+    aq = kt["act_quant"]
+    act_quant = {"bound": "hbm", "kernel": q_kernel, "achieved": aq["achieved"], "peak": hbm, "unit": "GB/s",
+                 "frac": aq["frac"], "us": aq["us"], "us_stream_loop": aq["us_stream"],
+                 "frac_stream_loop": aq["frac_stream"], "bytes": aq["bytes"], "traffic": q_traffic,
+                 "peak_source": f"{src} copy bandwidth",
+                 "timing": "fp8q_quant_act with both scale layouts, CUDA graph of back-to-back launches over "
+                           "rotating inputs > 3x L2"}
+    if m <= 64:
+        act_quant["variants"] = {v: aq[v] for v in ("single", "multi") if v in aq}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -503,11 +670,12 @@ def ours_arm(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
             "config": {"workload": args.workload, "m": m, "n": n, "k": k, "parallelism": f"replicas{world}",
                        "weight_format": args.weight_format, "decode_path": args.decode_path,
-                       "l2": f"{N_SETS} rotating input sets ({N_SETS * (m * k * 2 + n * k + m * n * 2) / 1e6:.0f} MB) > L2"},
+                       "l2": f"{n_sets} rotating input sets ({n_sets * (m * k * 3 + n * k + m * n * 2) / 1e6:.0f} MB) "
+                             f"for the step; kernel loops rotate > 3x L2"},
             "roofline": roofline,
-            "act_quant": {"bound": "hbm", "kernel": q_kernel, "achieved": quant_gbs, "peak": hbm, "unit": "GB/s",
-                          "frac": quant_gbs / hbm, "us": quant_us, "bytes": quant_bytes(m, k), "traffic": q_traffic,
-                          "peak_source": f"{src} copy bandwidth"},
+            "act_quant": act_quant,
+            "linear_us": {"stream_loop": kt["linear"]["us_stream"], "graph": kt["linear"]["us_graph"]},
+            "per_config": per_config,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": m * k * 2,
                     "d2h_bytes_per_step": m * n * 2},
@@ -571,6 +739,8 @@ def ffn_reference_arm(args):
         "impl": "reference", "metric": FFN_METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": flops / (value * 1e12) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step_kind": f"extrapolated: each step times {rows} of {m} token rows and scales that time "
+                            f"to the whole step",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "m": m, "d": d, "i": i},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
@@ -725,6 +895,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(FFN_WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only the chosen workload's kernels, not the other configurations")
     ap.add_argument("--weight-format", choices=["block128", "per_row"], default="block128",
                     help="weight scales per 128x128 block (the pages' format) or one per weight row")
     ap.add_argument("--decode-path", choices=["two_launch", "fused"], default="two_launch",

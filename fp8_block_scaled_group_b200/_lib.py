@@ -54,6 +54,7 @@ SIGNATURES = {
     "fp8q_linear_scale_offset": (SZ, [U32, U32]),
     "fp8q_linear": (ctypes.c_int, [P, P, P, P, P, SZ, U32, U32, U32, P]),
     "fp8q_linear_noalloc": (ctypes.c_int, [P, P, P, P, U32, U32, U32, P]),
+    "fp8q_diag_stalled_linear": (ctypes.c_int, [P, P, P, P, P, SZ, U32, U32, U32, ctypes.c_uint64, P]),
     "fp8q_silu_mul_quant": (ctypes.c_int, [P, P, U32, P, P, P, U32, U32, P]),
     "fp8q_ffn_workspace_layout": (ctypes.c_int, [U32, U32, U32, ctypes.POINTER(SZ)]),
     "fp8q_ffn_workspace_bytes": (SZ, [U32, U32, U32]),

@@ -341,12 +341,13 @@ def convert_e4m3(t: torch.Tensor, stream=None) -> torch.Tensor:
     return out
 
 
-def check_division(stream=None) -> tuple[int, int, int]:
-    """Run the exhaustive division check; returns (pairs, code mismatches, quotient mismatches)."""
-    counts = torch.zeros(3, dtype=torch.int64, device="cuda")
+def check_division(stream=None) -> tuple[int, int, int, int]:
+    """Run the exhaustive division check; returns (pairs, code mismatches,
+    quotient mismatches, scale or reciprocal mismatches)."""
+    counts = torch.zeros(4, dtype=torch.int64, device="cuda")
     _lib.check(_lib.load().fp8q_check_division(_p(counts), _stream(stream)), "fp8q_check_division")
-    a, b, c = counts.cpu().tolist()
-    return int(a), int(b), int(c)
+    a, b, c, d = counts.cpu().tolist()
+    return int(a), int(b), int(c), int(d)
 
 
 def launch_count() -> int:

@@ -10,6 +10,7 @@
 #include "fp8q.h"
 #include "internal.h"
 #include "nvfp4.h"
+#include "ptx.cuh"
 
 namespace fp8q {
 
@@ -167,16 +168,18 @@ fp8q_status fp8q_quant_pick(uint32_t m, uint32_t k, uint32_t sm_count, int32_t r
     const uint32_t G = k / kGroup;
     fp8q_quant_pick_t p;
     std::memset(&p, 0, sizeof p);
-    const uint64_t multi = static_cast<uint64_t>(ceil_div(G, kMultiGroupsPerCta)) * ceil_div(m, kMultiRowsPerCta);
-    p.multi_ctas = static_cast<uint32_t>(multi > 0xFFFFFFFFull ? 0xFFFFFFFFull : multi);
+    // m * G < 2^24 for every m*k < 2^31 the quantizer accepts; larger
+    // products are only ever asked for by the pick itself.
+    const uint64_t groups = static_cast<uint64_t>(m) * G;
+    const uint64_t stages = (groups + kStreamChunkGroups - 1) / kStreamChunkGroups;
+    const uint64_t cap = static_cast<uint64_t>(sm_count) * kStreamCtasPerSm;
+    p.multi_ctas = static_cast<uint32_t>(stages < cap ? stages : cap);
     p.floor_ctas = static_cast<uint32_t>(floor_cta_count(sm_count, kMultiMinCtasPerSm));
     int32_t v;
     if (requested == FP8Q_QUANT_AUTO) {
-        // The floor, read from the same function the tests and logs use, so
-        // it cannot disagree with the grid it guards.
-        const uint32_t min_m =
-            fp8q_quant_floor_min_m(k, sm_count, kMultiGroupsPerCta, kMultiRowsPerCta, kMultiMinCtasPerSm);
-        v = m >= min_m ? FP8Q_QUANT_MULTI : FP8Q_QUANT_SINGLE;
+        // The pages' rule: the multi-group kernel only when its grid reaches
+        // the CTA-count floor.
+        v = p.multi_ctas >= p.floor_ctas ? FP8Q_QUANT_MULTI : FP8Q_QUANT_SINGLE;
     } else {
         v = requested;
         p.forced = 1;
@@ -184,10 +187,11 @@ fp8q_status fp8q_quant_pick(uint32_t m, uint32_t k, uint32_t sm_count, int32_t r
     p.variant = v;
     if (v == FP8Q_QUANT_MULTI) {
         p.grid_x = p.multi_ctas;
-        p.block_x = 64;
-        p.groups_per_cta = kMultiGroupsPerCta * kMultiRowsPerCta;
+        p.block_x = kStreamThreads;
+        const uint64_t per_cta = p.multi_ctas ? (stages + p.multi_ctas - 1) / p.multi_ctas : 0;
+        p.groups_per_cta = static_cast<uint32_t>(per_cta * kStreamChunkGroups);
     } else {
-        const uint64_t single = static_cast<uint64_t>(G) * m;
+        const uint64_t single = groups;
         p.grid_x = static_cast<uint32_t>(single > 0xFFFFFFFFull ? 0xFFFFFFFFull : single);
         p.block_x = 16;
         p.groups_per_cta = 1;
@@ -207,7 +211,7 @@ fp8q_status fp8q_quant_act_variant(const void* x, void* q, float* s_row, float* 
     fp8q_quant_pick_t pick;
     if ((st = fp8q_quant_pick(m, k, static_cast<uint32_t>(dev.sms), variant, &pick)) != FP8Q_OK) return st;
     log_pick(pick, m, k);
-    QuantLaunch L{x, q, s_row, s_kmajor, m, k, fp8q_m_pad(m), pick.variant};
+    QuantLaunch L{x, q, s_row, s_kmajor, m, k, fp8q_m_pad(m), pick.variant, static_cast<uint32_t>(dev.sms)};
     return from_cuda(launch_quant_act(L, static_cast<cudaStream_t>(stream)));
 }
 
@@ -306,6 +310,32 @@ fp8q_status fp8q_linear_decode_fused(const void* x, const void* wq, const float*
     if ((st = current_device(&dev)) != FP8Q_OK) return st;
     GemmLaunch L{ws, s_k, wq, w_scale, y, m, n, k, fp8q_m_pad(m), false, weight_format == FP8Q_WEIGHT_PER_ROW, x};
     return from_cuda(launch_gemm(L, static_cast<cudaStream_t>(stream)));
+}
+
+fp8q_status fp8q_diag_stalled_linear(const void* x, const void* wq, const float* w_scale, void* y, void* workspace,
+                                     size_t workspace_bytes, uint32_t m, uint32_t n, uint32_t k,
+                                     uint64_t wait_budget_cycles, void* stream) {
+    if (wait_budget_cycles == 0 || wait_budget_cycles > static_cast<uint64_t>(kWaitBudgetCycles)) return FP8Q_ERR_ARG;
+    if (k == 0 || k % kGroup || n == 0 || n % kGroup) return FP8Q_ERR_SHAPE;
+    if (m == 0) return FP8Q_OK;
+    if (!x || !wq || !w_scale || !y || !workspace) return FP8Q_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FP8Q_ERR_WORKSPACE;
+    if (workspace_bytes < fp8q_linear_workspace_bytes(m, k)) return FP8Q_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* s_k = reinterpret_cast<float*>(ws + fp8q_linear_scale_offset(m, k));
+    fp8q_status st = check_quant_args(x, ws, nullptr, s_k, m, k);
+    if (st != FP8Q_OK) return st;
+    if ((st = check_gemm_args(ws, s_k, wq, w_scale, y, m, n, k)) != FP8Q_OK) return st;
+    DeviceInfo dev;
+    if ((st = current_device(&dev)) != FP8Q_OK) return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const long long budget = static_cast<long long>(wait_budget_cycles);
+    QuantLaunch Lq{x, ws, nullptr, s_k, m, k, fp8q_m_pad(m), kVariantMulti, static_cast<uint32_t>(dev.sms)};
+    Lq.diag_budget = budget;
+    if ((st = from_cuda(launch_quant_act(Lq, s))) != FP8Q_OK) return st;
+    GemmLaunch Lg{ws, s_k, wq, w_scale, y, m, n, k, fp8q_m_pad(m), false, false};
+    Lg.diag_budget = budget;
+    return from_cuda(launch_gemm(Lg, s));
 }
 
 fp8q_status fp8q_linear(const void* x, const void* wq, const float* w_scale, void* y, void* workspace,
@@ -524,13 +554,14 @@ fp8q_status fp8q_device_error(void* stream, uint32_t* code) {
     DeviceInfo dev;
     fp8q_status st = current_device(&dev);
     if (st != FP8Q_OK) return st;
-    uint32_t nvfp4_code = 0;
+    uint32_t nvfp4_code = 0, quant_code = 0;
     if (read_clear_device_error(code, static_cast<cudaStream_t>(stream)) != cudaSuccess ||
-        read_clear_nvfp4_error(&nvfp4_code, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        read_clear_nvfp4_error(&nvfp4_code, static_cast<cudaStream_t>(stream)) != cudaSuccess ||
+        read_clear_quant_error(&quant_code, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
         cudaGetLastError();
         return FP8Q_ERR_CUDA;
     }
-    *code |= nvfp4_code;
+    *code |= nvfp4_code | quant_code;
     return *code ? FP8Q_ERR_DEVICE_TIMEOUT : FP8Q_OK;
 }
 

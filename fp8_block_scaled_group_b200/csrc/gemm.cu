@@ -100,6 +100,8 @@ struct Shape {
     uint32_t M, N, G, Mp;
     uint32_t num_m, num_tiles;
     uint32_t w_per_row;  // weight scales: 0 = [N/128, K/128] blocks, 1 = one per weight row [N]
+    uint32_t no_copies;  // timeout diagnostics: the producer issues no copies
+    long long budget;    // clock budget of every wait
 };
 
 __device__ __forceinline__ void tile_coords(const Shape& sh, uint32_t tile, uint32_t& m0, uint32_t& n0) {
@@ -181,7 +183,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     if (warp < 4) {
         regs_dec<kRegsLow>();
-        if (warp == 0 && lane == 0) {
+        if (warp == 0 && lane == 0 && !sh.no_copies) {
             // Set-up above overlaps the producing kernel (quantizer) when
             // launched as its dependent; its outputs are read from here on.
             grid_dependency_wait();
@@ -195,14 +197,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 for (uint32_t kb = 0; kb < G; ++kb, ++it) {
                     const uint32_t s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
-                    if (!mbar_wait(&sm.empty[s], ph ^ 1u, abort)) {
+                    if (!mbar_wait(&sm.empty[s], ph ^ 1u, abort, sh.budget)) {
                         ok = false;
                         break;
                     }
                     if constexpr (!kDirect) {
                         const uint32_t ss = it % kScaleStages;
                         const uint32_t sph = (it / kScaleStages) & 1u;
-                        if (!mbar_wait(&sm.sempty[ss], sph ^ 1u, abort)) {
+                        if (!mbar_wait(&sm.sempty[ss], sph ^ 1u, abort, sh.budget)) {
                             ok = false;
                             break;
                         }
@@ -237,12 +239,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t ph = (it / kStages) & 1u;
                     const uint32_t b = it & 1u;
                     const uint32_t tph = (it >> 1) & 1u;
-                    if (!mbar_wait(&sm.full[s], ph, abort)) {
+                    if (!mbar_wait(&sm.full[s], ph, abort, sh.budget)) {
                         ok = false;
                         break;
                     }
                     sm.consumed[par] = it + 1;
-                    if (!mbar_wait(&sm.tempty[b], tph ^ 1u, abort)) {
+                    if (!mbar_wait(&sm.tempty[b], tph ^ 1u, abort, sh.budget)) {
                         ok = false;
                         break;
                     }
@@ -319,7 +321,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     aq3 = row_ok && kb + 4 < G ? __ldg(a_row + static_cast<size_t>(kb + 4) * sh.Mp) : 0.0f;
                 }
                 if (!per_row && kb + 1 < G) w_next = __ldg(ws_row + kb + 1);
-                const bool got = (kDirect || mbar_wait(&sm.sfull[ss], sph, abort)) && mbar_wait(&sm.tfull[b], tph, abort);
+                const bool got = (kDirect || mbar_wait(&sm.sfull[ss], sph, abort, sh.budget)) && mbar_wait(&sm.tfull[b], tph, abort, sh.budget);
                 if (!__all_sync(0xFFFFFFFFu, got)) {
                     ok = false;
                     break;
@@ -469,6 +471,8 @@ constexpr size_t decode_smem_bytes() {
 struct DecodeShape {
     uint32_t M, N, G, split, Mp;
     uint32_t w_per_row;  // weight scales: 0 = [N/128, K/128] blocks, 1 = one per weight row [N]
+    uint32_t no_copies;  // timeout diagnostics: the producer issues no copies
+    long long budget;    // clock budget of every wait
 };
 
 template <uint32_t NT>
@@ -563,13 +567,13 @@ __global__ void __launch_bounds__(FUSE ? kDecFusedThreads : kDecThreads, 2)
     const uint32_t r_local = (warp & 3u) * 32u + lane;  // weight row within the slice
 
     if (warp == 0) {
-        if (lane == 0) {
+        if (lane == 0 && !sh.no_copies) {
             grid_dependency_wait();
             for (uint32_t it = 0; it < nk; ++it) {
                 const uint32_t kb = kb0 + it;
                 const uint32_t s = it % kDecStages;
                 const uint32_t ph = (it / kDecStages) & 1u;
-                if (!mbar_wait(&sm.empty[s], ph ^ 1u, abort)) break;
+                if (!mbar_wait(&sm.empty[s], ph ^ 1u, abort, sh.budget)) break;
                 if (FUSE) {
                     mbar_arrive_expect_tx(&sm.full[s], BM * BK);
                     tma_load_2d(sm.w[s], &tmW, &sm.full[s], static_cast<int32_t>(kb * BK), static_cast<int32_t>(n0));
@@ -590,9 +594,9 @@ __global__ void __launch_bounds__(FUSE ? kDecFusedThreads : kDecThreads, 2)
                 const uint32_t ph = (it / kDecStages) & 1u;
                 const uint32_t b = it % kDecBufs;
                 const uint32_t tph = (it / kDecBufs) & 1u;
-                if (!mbar_wait(&sm.full[s], ph, abort)) break;
+                if (!mbar_wait(&sm.full[s], ph, abort, sh.budget)) break;
                 sm.consumed = it + 1;
-                if (!mbar_wait(&sm.tempty[b], tph ^ 1u, abort)) break;
+                if (!mbar_wait(&sm.tempty[b], tph ^ 1u, abort, sh.budget)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + b * NT;
                 const uint64_t ad = smem_desc_k_sw128(smem_addr(sm.w[s]));
@@ -620,7 +624,7 @@ __global__ void __launch_bounds__(FUSE ? kDecFusedThreads : kDecThreads, 2)
             const uint32_t tph = (it / kDecBufs) & 1u;
             const float wsc = w_next;
             if (!per_row && it + 1 < nk) w_next = __ldg(ws_row + kb0 + it + 1);
-            const bool got = mbar_wait(&sm.tfull[b], tph, abort);
+            const bool got = mbar_wait(&sm.tfull[b], tph, abort, sh.budget);
             if (!__all_sync(0xFFFFFFFFu, got)) break;
             tc_fence_after();
             uint32_t v[NT];
@@ -669,7 +673,7 @@ __global__ void __launch_bounds__(FUSE ? kDecFusedThreads : kDecThreads, 2)
             const uint32_t s = it % kDecStages;
             const uint32_t ph = (it / kDecStages) & 1u;
             if (it + 1 < nk) load_block(kb + 1, nxt);
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.empty[s], ph ^ 1u, abort))) break;
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.empty[s], ph ^ 1u, abort, sh.budget))) break;
 #pragma unroll
             for (uint32_t r = 0; r < R; ++r) {
                 const uint32_t t = gi + 8u * r;
@@ -882,6 +886,8 @@ cudaError_t launch_decode(const GemmLaunch& L, int sms, cudaStream_t stream) {
     sh.G = L.k / BK;
     sh.Mp = L.mp;
     sh.w_per_row = L.w_per_row ? 1u : 0u;
+    sh.no_copies = L.diag_budget != 0 ? 1u : 0u;
+    sh.budget = L.diag_budget != 0 ? L.diag_budget : kWaitBudgetCycles;
     const uint32_t slices = L.n / BM;
     const uint32_t split = decode_split(slices, sh.G, sms);
     sh.split = split;
@@ -928,6 +934,8 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream) {
     sh.num_m = (L.m + BM_PAIR - 1) / BM_PAIR;
     sh.num_tiles = sh.num_m * ((L.n + BN - 1) / BN);
     sh.w_per_row = L.w_per_row ? 1u : 0u;
+    sh.no_copies = L.diag_budget != 0 ? 1u : 0u;
+    sh.budget = L.diag_budget != 0 ? L.diag_budget : kWaitBudgetCycles;
     const uint32_t max_pairs = static_cast<uint32_t>(ks.sms) / 2;
     const uint32_t grid = 2 * (sh.num_tiles < max_pairs ? sh.num_tiles : max_pairs);
     cudaLaunchConfig_t cfg = {};

@@ -46,38 +46,79 @@ __device__ __forceinline__ float absmax8_bits(const uint4 v) {
     return __uint_as_float((hi > lo ? hi : lo) << 16);
 }
 
-// The scale of a group with absolute maximum `amax`: one fp32 division.
+// The scale of a group with absolute maximum `amax`: RN(max(amax, 1e-10)/448),
+// the correctly rounded fp32 quotient, formed with Markstein's correction
+// (P. Markstein, IBM J. Res. Dev. 34(1), 1990) from c = RN(1/448):
+//   q0 = RN(a c),  e = RN(a - 448 q0) (exact with a fused multiply-add),
+//   s  = RN(q0 + e c).
+// amax is the largest |x| of a group of bf16 values, so a takes at most
+// 20645 distinct values (1e-10 and the bf16 values above it);
+// fp8q_check_division compares this with IEEE division on every one of them.
+constexpr float kInv448 = 0x1.24924ap-9f;  // RN(1/448)
 __device__ __forceinline__ float group_scale(float amax) {
-    return __fdiv_rn(fmaxf(amax, 1e-10f), 448.0f);
+    const float a = fmaxf(amax, 1e-10f);
+    const float q0 = __fmul_rn(a, kInv448);
+    const float e = __fmaf_rn(-q0, 448.0f, a);
+    return __fmaf_rn(e, kInv448, q0);
 }
 
-// x / s for a pair of values, rounded to nearest even, from the correctly
-// rounded reciprocal r = RN(1/s) and one remainder correction (Markstein's
+// -RN(1/s) for a group scale s: the hardware reciprocal approximation
+// (rcp.approx, within an ulp) refined by one Newton-Raphson step with a
+// fused multiply-add, r = r0 + r0 (1 - s r0), then negated. Group scales
+// take at most 20645 values (see group_scale), and fp8q_check_division
+// compares this with the correctly rounded reciprocal on every one of them.
+__device__ __forceinline__ float neg_recip(float s) {
+    float r0;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(s));
+    const float e = __fmaf_rn(-s, r0, 1.0f);
+    return -__fmaf_rn(r0, e, r0);
+}
+
+// The negated quotient -(x / s) for a pair of values, rounded to nearest
+// even, from nr = -RN(1/s) and one remainder correction (Markstein's
 // division scheme, P. Markstein, IBM J. Res. Dev. 34(1), 1990):
-//   q0 = RN(x * r),  e = RN(x - q0 * s) (exact with a fused multiply-add),
-//   q  = RN(q0 + e * r).
-// The sign of x is put back at the end so that -0 stays -0. For every pair
-// (x, amax) of bf16 values with |x| <= amax, the code this gives equals the
-// code of the IEEE quotient: fp8q_check_division verifies it exhaustively on
-// the device.
-__device__ __forceinline__ float2 div2_by_scale(float2 x, float s, float r) {
-    const float2 q0 = __fmul2_rn(x, make_float2(r, r));
-    const float2 e = __ffma2_rn(make_float2(-q0.x, -q0.y), make_float2(s, s), x);
-    const float2 q = __ffma2_rn(e, make_float2(r, r), q0);
-    return make_float2(__uint_as_float(__float_as_uint(q.x) | (__float_as_uint(x.x) & 0x80000000u)),
-                       __uint_as_float(__float_as_uint(q.y) | (__float_as_uint(x.y) & 0x80000000u)));
+//   q0 = RN(x * nr) = -RN(x / s approx.),
+//   e  = RN(q0 * s + x)   (the exact remainder, with a fused multiply-add),
+//   q  = RN(e * nr + q0).
+// Every step is the negation of the scheme run on +r, because rounding to
+// nearest is symmetric, so q is exactly -(the scheme's quotient) for x != 0.
+// For x = +-0 the zeros come out with the sign of -x (-0 + +0 = +0 in round
+// to nearest), so negating the result's code gives the code of a zero with
+// the sign of x, with no per-element sign repair. For every pair (x, amax) of
+// bf16 values with |x| <= amax, the code this gives, sign-flipped, equals the
+// code of the IEEE quotient x / s: fp8q_check_division verifies it
+// exhaustively on the device.
+__device__ __forceinline__ float2 neg_div2_by_scale(float2 x, float s, float nr) {
+    const float2 q0 = __fmul2_rn(x, make_float2(nr, nr));
+    const float2 e = __ffma2_rn(q0, make_float2(s, s), x);
+    return __ffma2_rn(e, make_float2(nr, nr), q0);
 }
 
-// 8 values / s -> 8 codes packed little-endian.
-__device__ __forceinline__ uint2 encode8(const float (&f)[8], float s) {
-    const float r = __frcp_rn(s);
+// e4m3 codes of -v are those of v with the sign bit flipped (round to
+// nearest even and saturation to +-448 are symmetric); four codes per word.
+constexpr uint32_t kCodeSignBits = 0x80808080u;
+
+// 8 values / s -> 8 codes packed little-endian, given nr = -RN(1/s).
+__device__ __forceinline__ uint2 encode8_nr(const float (&f)[8], float s, float nr) {
     uint32_t c[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const float2 q = div2_by_scale(make_float2(f[2 * i], f[2 * i + 1]), s, r);
+        const float2 q = neg_div2_by_scale(make_float2(f[2 * i], f[2 * i + 1]), s, nr);
         c[i] = cvt_e4m3x2(q.x, q.y);
     }
-    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+    return make_uint2((c[0] | (c[1] << 16)) ^ kCodeSignBits, (c[2] | (c[3] << 16)) ^ kCodeSignBits);
+}
+
+__device__ __forceinline__ uint2 encode8(const float (&f)[8], float s) {
+    return encode8_nr(f, s, neg_recip(s));
+}
+
+// max(|a|, |b|) of two pairs of packed bf16 per half (the sign bit of each
+// result half is the xor of the inputs' signs: clear it before use).
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
 }
 
 // Let a dependent kernel (the GEMM of a fused linear, launched with

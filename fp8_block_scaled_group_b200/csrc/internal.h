@@ -11,14 +11,23 @@ namespace fp8q {
 constexpr int kVariantSingle = 1;
 constexpr int kVariantMulti = 2;
 
-// MULTI geometry: 8 K-groups per CTA (eight lanes each), each quantized
-// for kMultiRowsPerCta consecutive tokens.
-constexpr uint32_t kMultiGroupsPerCta = 8;
-constexpr uint32_t kMultiRowsPerCta = 4;
-// MULTI runs when its grid reaches this many CTAs per SM (B200 sweep of
-// both variants over M in 1..4576 at K = 5120, 6144, 17408: MULTI overtakes
-// SINGLE once its grid holds about two thirds of a CTA per SM).
-constexpr float kMultiMinCtasPerSm = 2.0f / 3.0f;
+// MULTI geometry (the streaming quantizer): every warp streams chunks of 16
+// groups (4 KB of X) through its own ring of 2 shared-memory slots and a
+// 2 KB code staging buffer; 7 warps a CTA, up to 3 CTAs per SM.
+constexpr uint32_t kStreamChunkGroups = 16;
+constexpr uint32_t kStreamSlots = 2;
+constexpr uint32_t kStreamWarps = 7;
+constexpr uint32_t kStreamThreads = 32 * kStreamWarps;
+constexpr uint32_t kStreamCtasPerSm = 3;
+// MULTI runs when its grid (one CTA per chunk, at most kStreamCtasPerSm per
+// SM) holds at least this many CTAs per SM; below it the one-group-per-CTA
+// kernel's many small CTAs finish sooner. From a B200 sweep of both variants
+// over M in 1..4576 at K = 5120, 6144, 17408: SINGLE was faster up to 63
+// MULTI CTAs and MULTI from 68 on, so the floor is ceil(0.45 * 148) = 67.
+constexpr float kMultiMinCtasPerSm = 0.45f;
+
+// CTAs of the MULTI grid for (m, k) on `sms` SMs.
+uint32_t stream_grid(uint32_t m, uint32_t k, uint32_t sms);
 
 struct QuantLaunch {
     const void* x;
@@ -27,6 +36,10 @@ struct QuantLaunch {
     float* s_k;
     uint32_t m, k, mp;
     int variant;
+    uint32_t sms;  // SMs of the device (sizes the MULTI grid)
+    // Timeout diagnostics only (0 in normal use): the MULTI kernel issues
+    // no copies and bounds each wait by this many clocks.
+    long long diag_budget = 0;
 };
 
 cudaError_t launch_quant_act(const QuantLaunch& L, cudaStream_t stream);
@@ -49,6 +62,9 @@ struct GemmLaunch {
     // Non-null (m <= 32 only): the bf16 activation [m, k]; the decode kernel
     // quantizes it itself and writes q and the K-major s_k as outputs.
     const void* x = nullptr;
+    // Timeout diagnostics only (0 in normal use): the kernel's producer
+    // issues no copies and each wait is bounded by this many clocks.
+    long long diag_budget = 0;
 };
 
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream);
@@ -69,6 +85,7 @@ cudaError_t launch_silu_mul_quant(const SiluLaunch& L, bool pdl, cudaStream_t st
 cudaError_t launch_check_silu_mul(unsigned long long* counts, uint32_t* max_err_bits, cudaStream_t stream);
 
 cudaError_t read_clear_device_error(uint32_t* code, cudaStream_t stream);
+cudaError_t read_clear_quant_error(uint32_t* code, cudaStream_t stream);
 
 void note_launch();
 

@@ -9,9 +9,15 @@
 // fp8q_linear on it.
 //
 // In host code `g_linear_scratch` is only a host-side stand-in for the
-// device array, not a device address; its device address is looked up with
-// cudaGetSymbolAddress once per device (with that device current) and that
-// address is what the kernels receive.
+// device array, not a device address. Its device address is looked up with
+// cudaGetSymbolAddress, with the device current, and that address is what
+// the kernels receive. The lookup is cached per device together with the
+// unique ID of the CUDA context it was made in; a call that finds a
+// different context current (for example after cudaDeviceReset made a new
+// primary context) looks the address up again instead of reusing one that
+// belonged to the old context.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "fp8q.h"
@@ -23,17 +29,61 @@ namespace {
 // The scratch holds the FP8 activation [M, K] and the K-major scales
 // [K/128, ceil16(M)] of one call (fp8q_linear_workspace_bytes(M, K)).
 // 16 MiB covers, e.g., M = 1168 tokens at K = 5120 (6.2 MB) or M = 900 at
-// K = 17408. Every GPU that loads the library holds this array until the
-// process exits.
+// K = 17408 (16.2 MB). Every GPU that loads the library holds this array
+// until the process exits.
 constexpr size_t kScratchBytes = size_t(16) << 20;
 
 static __device__ __align__(256) uint8_t g_linear_scratch[kScratchBytes];
 
-std::mutex g_scratch_mu;
-void* g_scratch_addr[64] = {};
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
-// Device address of g_linear_scratch on the current device, looked up on the
-// first call made on that device.
+struct DriverFns {
+    CtxGetCurrentFn get_current = nullptr;
+    CtxGetIdFn get_id = nullptr;
+};
+
+const DriverFns& driver_fns() {
+    static DriverFns fns;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fns.get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fns.get_id = reinterpret_cast<CtxGetIdFn>(p);
+        cudaGetLastError();
+    });
+    return fns;
+}
+
+// ID of the context current on this thread, or 0 if there is none yet (the
+// runtime makes the primary context current on its first call that needs one).
+unsigned long long current_context_id() {
+    const DriverFns& f = driver_fns();
+    if (!f.get_current || !f.get_id) return 0;
+    CUcontext ctx = nullptr;
+    if (f.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    unsigned long long id = 0;
+    if (f.get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+struct ScratchEntry {
+    unsigned long long ctx_id = 0;
+    void* addr = nullptr;
+};
+
+std::mutex g_scratch_mu;
+ScratchEntry g_scratch[64];
+
+// Device address of g_linear_scratch in the current device's current context.
+// The first call in a context looks it up (and so should come before any
+// stream capture); later calls in the same context reuse it.
 fp8q_status scratch_address(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
@@ -48,16 +98,21 @@ fp8q_status scratch_address(void** out) {
     }
     if (major != 10 || minor != 0) return FP8Q_ERR_UNSUPPORTED_DEVICE;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
+    ScratchEntry& e = g_scratch[dev];
+    const unsigned long long id = current_context_id();
+    if (e.addr == nullptr || id == 0 || id != e.ctx_id) {
         void* p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_linear_scratch);
-        if (e != cudaSuccess || p == nullptr) {
+        const cudaError_t err = cudaGetSymbolAddress(&p, g_linear_scratch);
+        if (err != cudaSuccess || p == nullptr) {
             cudaGetLastError();
+            e = ScratchEntry{};
             return FP8Q_ERR_CUDA;
         }
-        g_scratch_addr[dev] = p;
+        // The lookup made the device's primary context current if it was not.
+        e.ctx_id = current_context_id();
+        e.addr = p;
     }
-    *out = g_scratch_addr[dev];
+    *out = e.addr;
     return FP8Q_OK;
 }
 

@@ -1,6 +1,6 @@
 // Inline-PTX building blocks for the NVFP4 kernels on sm_100a: the e4m3
-// value of a code, the packed E2M1 conversion, untiled bulk loads, the
-// scale-factor copy into TMEM and the block-scaled MMA (kind::mxf4nvf4).
+// value of a code, the packed E2M1 conversion, the scale-factor copy into
+// TMEM and the block-scaled MMA (kind::mxf4nvf4).
 #pragma once
 
 #include "ptx.cuh"
@@ -35,15 +35,6 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
 }
 
 // ------------------------------------------- block-scaled NVFP4 (MMA) --
-
-// Untiled bulk copy of `bytes` from global to shared memory (both addresses
-// 16-byte aligned, a multiple of 16 bytes), completion counted on `bar`.
-__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     smem_addr(smem_dst)),
-                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
-                 : "memory");
-}
 
 // Shared-memory descriptor of one scale-factor atom: 32 rows of 16 bytes,
 // contiguous, read as four 8-row core matrices 128 bytes apart (stride

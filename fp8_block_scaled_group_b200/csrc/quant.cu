@@ -5,39 +5,53 @@
 // per token and per 128-wide K group, amax = max |x|, s = max(amax, 1e-10)/448
 // (IEEE fp32 division), q = e4m3 RNE-satfinite of x/s (IEEE fp32 division).
 //
-// Both activation variants are one HBM stream. In SINGLE a 128-element group
-// is owned by 16 lanes holding 8 bf16 each (one 16-byte load), in MULTI by 8
-// lanes holding 16; amax is reduced with xor-shuffles inside those lanes and
-// each lane stores its codes as 8-byte stores, so a group's 128 codes leave
-// as contiguous runs.
 // The scale goes to the row-major [M, K/128] buffer and, in the same kernel,
 // to the K-major [K/128, ceil16(M)] buffer, whose pad rows the same launch
 // zero-fills; the pages spend a separate transpose launch on that layout
 // (`fp8_act_scale_to_kmajor`).
 //
-//   SINGLE: one group per CTA (16 threads), grid (K/128, M).
-//   MULTI : 8 consecutive groups of RPC consecutive tokens per CTA
-//           (64 threads, 8 lanes per group), grid (ceil((K/128)/8),
-//           ceil(M/RPC)). Each lane keeps 2*RPC independent 16-byte loads
-//           in flight.
+//   SINGLE: one group per CTA (16 threads, 16 bytes each), 1-D grid of M*G
+//           CTAs: many small CTAs, the lowest latency for decode widths.
+//   MULTI : a persistent streaming kernel. X [M, K] row-major is one
+//           contiguous run of M*G groups of 256 bytes, in (token, group)
+//           order, and so are the codes (128 bytes a group) and the
+//           row-major scales. The run is cut into stages of 32 groups (8 KB
+//           of X); CTA c takes stages c, c + C, c + 2C, ... A producer thread
+//           streams each stage into a shared-memory ring with one bulk copy
+//           (cp.async.bulk, completion counted on an mbarrier), up to
+//           kStreamSlots stages ahead, so an SM keeps up to 4 x 48 KB of X in
+//           flight from the kernel's first cycles. Eight consumer warps each
+//           quantize 4 groups of every stage (8 lanes per group, 16 elements
+//           a lane) and store codes and scales directly.
 #include <cuda_bf16.h>
 
 #include "group_quant.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
+#include <mutex>
+
 namespace fp8q {
 
-// SINGLE: blockDim 16, grid (G, M): CTA (g, t) quantizes group g of token t.
+// Device error word of the activation quantizer (bit 2 of fp8q_device_error):
+// a streaming CTA gave up on a bounded wait.
+__device__ uint32_t g_quant_error = 0;
+constexpr uint32_t kQuantErrorBit = 4u;
+
+// SINGLE: blockDim 16, 1-D grid of G*M CTAs: CTA b quantizes group b % G of
+// token b / G.
 __global__ void __launch_bounds__(16) quant_act_single_kernel(const uint16_t* __restrict__ x,
                                                              uint8_t* __restrict__ q, float* __restrict__ s_row,
                                                              float* __restrict__ s_k, uint32_t m, uint32_t k,
                                                              uint32_t mp) {
-    if (gridDim.x * gridDim.y <= kSingleTriggerMaxGrid) trigger_dependents();
-    const uint32_t G = gridDim.x;
-    const uint32_t g = blockIdx.x, t = blockIdx.y;
+    if (gridDim.x <= kSingleTriggerMaxGrid) trigger_dependents();
+    const uint32_t G = k >> 7;
+    const uint32_t t = blockIdx.x / G, g = blockIdx.x - t * G;
     const uint32_t lane = threadIdx.x;
     const size_t off = static_cast<size_t>(t) * k + static_cast<size_t>(g) * 128 + lane * 8;
+    // Nothing is read or written in global memory before the grid this
+    // launch may depend on has completed.
+    grid_dependency_wait();
     const uint4 v = ld_stream16(x + off);
     float f[8];
     widen8(v, f);
@@ -53,63 +67,157 @@ __global__ void __launch_bounds__(16) quant_act_single_kernel(const uint16_t* __
     zero_kmajor_pad(s_k, m, mp, G);
 }
 
-// MULTI: blockDim 64, grid (ceil(G/8), ceil(m/RPC)). Eight lanes own one
-// group: lane l holds elements 8l..8l+7 and 64+8l..64+8l+7 of it (two 16-byte
-// loads, each instruction covering the group's 128 contiguous bytes), so the
-// per-group work (scale, reciprocal, shuffles, scale stores) is shared by 16
-// elements per lane. Octet o of CTA (bx, by) owns group g = 8*bx + o for
-// tokens RPC*by .. RPC*by + RPC - 1; every load of the CTA is issued before
-// any arithmetic. Token validity is the same for the whole CTA, so rows past
-// m are skipped outright; a group past G (K/128 not a multiple of 8) computes
-// on zeros, so the shuffles still see their full warp, and stores nothing.
-template <int RPC>
-__global__ void __launch_bounds__(64) quant_act_multi_kernel(const uint16_t* __restrict__ x,
-                                                            uint8_t* __restrict__ q, float* __restrict__ s_row,
-                                                            float* __restrict__ s_k, uint32_t m, uint32_t k,
-                                                            uint32_t mp) {
-    if ((blockIdx.y * gridDim.x + blockIdx.x) + kMultiTriggerTail >= gridDim.x * gridDim.y) trigger_dependents();
+// MULTI (streaming). Every warp is an independent stream: its lane 0
+// bulk-copies chunks of kStreamChunkGroups groups (4 KB of X) into the
+// warp's own ring of kStreamSlots shared-memory slots, each completion
+// counted on the slot's own mbarrier, and the warp quantizes each chunk as
+// it lands, two lanes per group (64 elements a lane). The chunk's codes (2 KB,
+// contiguous in Q) are gathered in a shared-memory staging buffer and leave
+// with one bulk store, so every 128-byte line of Q is written whole. No warp
+// waits for another. Chunk c goes to CTA c % gridDim.x, warp
+// (c / gridDim.x) % kStreamWarps, so consecutive chunks are in flight on
+// different SMs.
+constexpr uint32_t kStreamChunkBytes = kStreamChunkGroups * 256;
+constexpr uint32_t kStreamCodeBytes = kStreamChunkGroups * 128;
+constexpr uint32_t kStreamWarpBytes = kStreamSlots * kStreamChunkBytes + kStreamCodeBytes;
+constexpr uint32_t kStreamSmemBytes = kStreamWarps * (kStreamWarpBytes + kStreamSlots * 8);
+static_assert(kStreamChunkGroups == 16, "two lanes per group, 32 lanes a chunk");
+
+// Bounded wait on one of this warp's barriers; false when the budget ran out.
+__device__ __forceinline__ bool warp_slot_wait(uint64_t* bar, uint32_t parity, long long budget) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > budget) return false;
+    return true;
+}
+
+__global__ void __launch_bounds__(kStreamThreads, kStreamCtasPerSm)
+    quant_act_stream_kernel(const uint16_t* __restrict__ x, uint8_t* __restrict__ q, float* __restrict__ s_row,
+                            float* __restrict__ s_k, uint32_t m, uint32_t k, uint32_t mp, long long budget,
+                            uint32_t no_copies) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint8_t* ring = smem + warp * kStreamWarpBytes;
+    uint8_t* codes = ring + kStreamSlots * kStreamChunkBytes;  // this warp's staging buffer
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStreamWarps * kStreamWarpBytes) + warp * kStreamSlots;
     const uint32_t G = k >> 7;
-    const uint32_t lane = threadIdx.x & 7;
-    const uint32_t g = blockIdx.x * 8 + (threadIdx.x >> 3);
-    const uint32_t t0 = blockIdx.y * RPC;
-    const bool g_ok = g < G;
-    const uint32_t rows = m - t0 < static_cast<uint32_t>(RPC) ? m - t0 : static_cast<uint32_t>(RPC);
-    uint4 v[RPC][2];
-#pragma unroll
-    for (int r = 0; r < RPC; ++r) {
-        if (g_ok && static_cast<uint32_t>(r) < rows) {
-            const uint16_t* src = x + static_cast<size_t>(t0 + r) * k + static_cast<size_t>(g) * 128 + lane * 8;
-            v[r][0] = ld_stream16(src);
-            v[r][1] = ld_stream16(src + 64);
-        } else {
-            v[r][0] = make_uint4(0u, 0u, 0u, 0u);
-            v[r][1] = make_uint4(0u, 0u, 0u, 0u);
-        }
+    const uint32_t total = m * G;  // groups; m*k < 2^31 keeps this below 2^24
+    const uint32_t chunks = (total + kStreamChunkGroups - 1) / kStreamChunkGroups;
+    const uint32_t first = blockIdx.x + gridDim.x * warp;
+    const uint32_t stride = gridDim.x * kStreamWarps;
+    const uint32_t mine = first < chunks ? (chunks - 1 - first) / stride + 1 : 0;
+
+    // Let the dependent (the GEMM of a fused linear) launch early.
+    trigger_dependents();
+    if (lane == 0) {
+        for (uint32_t i = 0; i < kStreamSlots; ++i) mbar_init(&full[i], 1);
+        fence_mbar_init();
     }
-#pragma unroll
-    for (int r = 0; r < RPC; ++r) {
-        if (static_cast<uint32_t>(r) >= rows) break;
-        const uint32_t t = t0 + r;
-        float amax = fmaxf(absmax8_bits(v[r][0]), absmax8_bits(v[r][1]));
-#pragma unroll
-        for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-        const float s = group_scale(amax);
-        float f0[8], f1[8];
-        widen8(v[r][0], f0);
-        widen8(v[r][1], f1);
-        const uint2 c0 = encode8(f0, s);
-        const uint2 c1 = encode8(f1, s);
-        if (g_ok) {
-            uint8_t* dst = q + static_cast<size_t>(t) * k + static_cast<size_t>(g) * 128 + lane * 8;
-            st_stream8(dst, c0);
-            st_stream8(dst + 64, c1);
-            if (lane == 0) {
-                if (s_row) s_row[static_cast<size_t>(t) * G + g] = s;
-                s_k[static_cast<size_t>(g) * mp + t] = s;
-            }
-        }
-    }
+    __syncwarp();
+    // Nothing is read or written in global memory before the grid this
+    // launch may depend on has completed.
+    grid_dependency_wait();
     zero_kmajor_pad(s_k, m, mp, G);
+
+    auto issue = [&](uint32_t i) {
+        const uint32_t slot = i % kStreamSlots;
+        const uint32_t g0 = (first + i * stride) * kStreamChunkGroups;
+        const uint32_t n = total - g0 < kStreamChunkGroups ? total - g0 : kStreamChunkGroups;
+        mbar_arrive_expect_tx(&full[slot], n * 256u);
+        bulk_load(ring + slot * kStreamChunkBytes, x + static_cast<size_t>(g0) * 128, n * 256u, &full[slot]);
+    };
+    uint32_t issued = 0;
+    if (lane == 0 && !no_copies) {
+        for (; issued < kStreamSlots && issued < mine; ++issued) issue(issued);
+    }
+
+    // Lane 2*gl + p owns half p of group gl of each chunk: 16-byte pieces
+    // c = 2j + p, j = 0..7 (elements 8c..8c+7), read in the order
+    // j = (i + gl) % 8 so that the eight lanes of every shared-memory phase
+    // touch eight different 16-byte columns of a 128-byte row.
+    const uint32_t gl = lane >> 1, p = lane & 1u;
+    bool ok = true;
+    uint32_t done = 0;
+    for (; done < mine; ++done) {
+        const uint32_t slot = done % kStreamSlots;
+        if (!__all_sync(0xFFFFFFFFu, warp_slot_wait(&full[slot], (done / kStreamSlots) & 1u, budget))) {
+            ok = false;
+            break;
+        }
+        const uint32_t g0 = (first + done * stride) * kStreamChunkGroups;
+        const uint32_t gf = g0 + gl;
+        const bool valid = gf < total;
+        uint4 v[8];
+        const uint8_t* src = ring + slot * kStreamChunkBytes + gl * 256u + p * 16u;
+#pragma unroll
+        for (uint32_t i = 0; i < 8; ++i)
+            v[i] = valid ? *reinterpret_cast<const uint4*>(src + ((i + gl) & 7u) * 32u) : make_uint4(0u, 0u, 0u, 0u);
+        // group amax: pairwise max of |bf16| over the 32 words, then the two
+        // halves, then the partner lane
+        uint32_t w[16];
+#pragma unroll
+        for (uint32_t i = 0; i < 4; ++i) {
+            w[4 * i + 0] = absmax_bf16x2(v[2 * i].x, v[2 * i + 1].x);
+            w[4 * i + 1] = absmax_bf16x2(v[2 * i].y, v[2 * i + 1].y);
+            w[4 * i + 2] = absmax_bf16x2(v[2 * i].z, v[2 * i + 1].z);
+            w[4 * i + 3] = absmax_bf16x2(v[2 * i].w, v[2 * i + 1].w);
+        }
+#pragma unroll
+        for (uint32_t n = 8; n > 0; n >>= 1)
+#pragma unroll
+            for (uint32_t i = 0; i < n; ++i) w[i] = absmax_bf16x2(w[i], w[i + n]);
+        const uint32_t hi = (w[0] >> 16) & 0x7FFFu, lo = w[0] & 0x7FFFu;
+        float amax = __uint_as_float((hi > lo ? hi : lo) << 16);
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+        // Every lane has read its pieces (the maximum used them all): the
+        // slot may be refilled with the chunk kStreamSlots ahead.
+        __syncwarp();
+        if (lane == 0 && issued < mine) {
+            fence_proxy_async_smem();
+            issue(issued++);
+        }
+        const float sc = group_scale(amax);
+        const float nr = neg_recip(sc);
+        uint2 c[8];
+#pragma unroll
+        for (uint32_t i = 0; i < 8; ++i) {
+            float f[8];
+            widen8(v[i], f);
+            c[i] = encode8_nr(f, sc, nr);
+        }
+        // The staging buffer is free once the previous chunk's bulk store
+        // has read it.
+        if (lane == 0) bulk_store_wait_read();
+        __syncwarp();
+        uint8_t* row = codes + gl * 128u + p * 8u;
+#pragma unroll
+        for (uint32_t i = 0; i < 8; ++i) *reinterpret_cast<uint2*>(row + ((i + gl) & 7u) * 16u) = c[i];
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            const uint32_t n = total - g0 < kStreamChunkGroups ? total - g0 : kStreamChunkGroups;
+            bulk_store(q + static_cast<size_t>(g0) * 128, codes, n * 128u);
+        }
+        if (valid && p == 0) {
+            if (s_row) s_row[gf] = sc;
+            const uint32_t t = gf / G;
+            s_k[static_cast<size_t>(gf - t * G) * mp + t] = sc;
+        }
+    }
+    if (!ok) {
+        // A wait ran out: report it, and let this warp's copies still in
+        // flight land (bounded) before the warp exits.
+        if (lane == 0) {
+            atomicOr(&g_quant_error, kQuantErrorBit);
+            for (uint32_t i = done; i < issued; ++i)
+                warp_slot_wait(&full[i % kStreamSlots], (i / kStreamSlots) & 1u, kWaitBudgetCycles);
+        }
+    }
+    // The codes are in global memory before the warp (and its CTA's shared
+    // memory) goes away.
+    if (lane == 0) bulk_store_wait_all();
+    __syncwarp();
 }
 
 // Weight blocks: grid (K/128, N/128), 256 threads. The block's 128 rows x
@@ -187,27 +295,35 @@ __global__ void convert_e4m3_kernel(const float* __restrict__ in, uint8_t* __res
 
 // Exhaustive check of the quantizers' division against IEEE division. CTA b
 // takes amax = the non-negative bf16 with bit pattern b (0 .. 0x7F7F, every
-// finite value), forms s = group_scale(amax) and, for every bf16 x with
-// |x| <= amax and both signs, compares the e4m3 code of div2_by_scale with
-// the code of __fdiv_rn(x, s), and the fp32 quotients themselves.
+// finite value). It checks the group scale and its negated reciprocal
+// against __fdiv_rn and __frcp_rn, then, for every bf16 x with |x| <= amax
+// and both signs, compares the sign-flipped e4m3 code of neg_div2_by_scale
+// with the code of the IEEE quotient __fdiv_rn(x, s), and the negated fp32
+// quotients with __fdiv_rn's.
 // counts[0] += pairs checked, counts[1] += code mismatches,
-// counts[2] += fp32 quotient mismatches.
+// counts[2] += fp32 quotient mismatches, counts[3] += amax values whose
+// scale or reciprocal differs from the IEEE one.
 __global__ void __launch_bounds__(256) check_division_kernel(unsigned long long* __restrict__ counts) {
     const uint32_t a_bits = blockIdx.x;
     const float amax = __uint_as_float(a_bits << 16);
     const float s = group_scale(amax);
-    const float r = __frcp_rn(s);
+    const float nr = neg_recip(s);
+    const float s_ieee = __fdiv_rn(fmaxf(amax, 1e-10f), 448.0f);
+    if (threadIdx.x == 0)
+        atomicAdd(&counts[3], static_cast<unsigned long long>((__float_as_uint(s) != __float_as_uint(s_ieee)) +
+                                                              (__float_as_uint(-nr) != __float_as_uint(__frcp_rn(s_ieee)))));
     unsigned long long pairs = 0, code_bad = 0, quot_bad = 0;
     for (uint32_t xb = threadIdx.x; xb <= a_bits; xb += blockDim.x) {
         const float xp = __uint_as_float(xb << 16);
         const float2 xv = make_float2(xp, -xp);
-        const float2 qf = div2_by_scale(xv, s, r);
-        const float qa = __fdiv_rn(xv.x, s), qb = __fdiv_rn(xv.y, s);
-        const uint16_t c_fast = cvt_e4m3x2(qf.x, qf.y);
+        const float2 qn = neg_div2_by_scale(xv, s, nr);
+        const float qa = __fdiv_rn(xv.x, s_ieee), qb = __fdiv_rn(xv.y, s_ieee);
+        const uint16_t c_fast = cvt_e4m3x2(qn.x, qn.y) ^ static_cast<uint16_t>(kCodeSignBits & 0xFFFFu);
         const uint16_t c_ieee = cvt_e4m3x2(qa, qb);
         pairs += 2;
         code_bad += ((c_fast & 0xFF) != (c_ieee & 0xFF)) + ((c_fast >> 8) != (c_ieee >> 8));
-        quot_bad += (__float_as_uint(qf.x) != __float_as_uint(qa)) + (__float_as_uint(qf.y) != __float_as_uint(qb));
+        quot_bad += ((__float_as_uint(qn.x) ^ 0x80000000u) != __float_as_uint(qa)) +
+                    ((__float_as_uint(qn.y) ^ 0x80000000u) != __float_as_uint(qb));
     }
     for (int o = 16; o > 0; o >>= 1) {
         pairs += __shfl_xor_sync(0xFFFFFFFFu, pairs, o);
@@ -223,19 +339,66 @@ __global__ void __launch_bounds__(256) check_division_kernel(unsigned long long*
 
 // ------------------------------------------------------------ launchers --
 
+uint32_t stream_grid(uint32_t m, uint32_t k, uint32_t sms) {
+    const uint32_t total = m * (k >> 7);
+    const uint32_t chunks = (total + kStreamChunkGroups - 1) / kStreamChunkGroups;
+    const uint32_t cap = sms * kStreamCtasPerSm;
+    return chunks < cap ? chunks : cap;
+}
+
 cudaError_t launch_quant_act(const QuantLaunch& L, cudaStream_t stream) {
     const uint32_t G = L.k >> 7;
+    // Both kernels wait for the grid before them (griddepcontrol.wait) before
+    // touching global memory, so they may launch as soon as that grid allows.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     if (L.variant == kVariantSingle) {
-        dim3 grid(G, L.m);
-        quant_act_single_kernel<<<grid, 16, 0, stream>>>(static_cast<const uint16_t*>(L.x), static_cast<uint8_t*>(L.q),
-                                                         L.s_row, L.s_k, L.m, L.k, L.mp);
-    } else {
-        dim3 grid((G + 7) / 8, (L.m + kMultiRowsPerCta - 1) / kMultiRowsPerCta);
-        quant_act_multi_kernel<kMultiRowsPerCta><<<grid, 64, 0, stream>>>(
-            static_cast<const uint16_t*>(L.x), static_cast<uint8_t*>(L.q), L.s_row, L.s_k, L.m, L.k, L.mp);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(G * L.m, 1, 1);
+        cfg.blockDim = dim3(16, 1, 1);
+        cfg.stream = stream;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, quant_act_single_kernel, static_cast<const uint16_t*>(L.x),
+                                                 static_cast<uint8_t*>(L.q), L.s_row, L.s_k, L.m, L.k, L.mp);
+        note_launch();
+        return e != cudaSuccess ? e : cudaGetLastError();
     }
+    static std::once_flag once[64];
+    static cudaError_t optin[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::call_once(once[dev], [dev] {
+        optin[dev] = cudaFuncSetAttribute(quant_act_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(kStreamSmemBytes));
+    });
+    if (optin[dev] != cudaSuccess) return optin[dev];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(stream_grid(L.m, L.k, L.sms), 1, 1);
+    cfg.blockDim = dim3(kStreamThreads, 1, 1);
+    cfg.dynamicSmemBytes = kStreamSmemBytes;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, quant_act_stream_kernel, static_cast<const uint16_t*>(L.x),
+                           static_cast<uint8_t*>(L.q), L.s_row, L.s_k, L.m, L.k, L.mp,
+                           L.diag_budget != 0 ? L.diag_budget : kWaitBudgetCycles,
+                           L.diag_budget != 0 ? 1u : 0u);
     note_launch();
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t read_clear_quant_error(uint32_t* code, cudaStream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return e;
+    uint32_t zero = 0;
+    e = cudaMemcpyFromSymbol(code, g_quant_error, sizeof(uint32_t));
+    if (e != cudaSuccess) return e;
+    if (*code) e = cudaMemcpyToSymbol(g_quant_error, &zero, sizeof(uint32_t));
+    return e;
 }
 
 cudaError_t launch_quant_weight(const void* w, void* wq, float* w_scale, uint32_t n, uint32_t k,
@@ -256,7 +419,7 @@ cudaError_t launch_quant_weight_rowwise(const void* w, void* wq, float* w_scale,
 }
 
 cudaError_t launch_check_division(unsigned long long* counts, cudaStream_t stream) {
-    cudaError_t e = cudaMemsetAsync(counts, 0, 3 * sizeof(unsigned long long), stream);
+    cudaError_t e = cudaMemsetAsync(counts, 0, 4 * sizeof(unsigned long long), stream);
     if (e != cudaSuccess) return e;
     check_division_kernel<<<0x7F80, 256, 0, stream>>>(counts);
     note_launch();

@@ -269,7 +269,9 @@ fp8q_status fp8q_linear_ex(const void *x, const void *wq, const float *w_scale,
  *     return FP8Q_ERR_WORKSPACE without enqueuing anything.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     before any stream capture. The address is cached with the ID of the
+ *     CUDA context it was found in, and looked up again when a call finds
+ *     another context current (after cudaDeviceReset, say).
  *   - Every call on a device shares the one array and it keeps the last
  *     call's contents; nothing in it needs clearing, because each call
  *     overwrites all of it that it reads. Calls that overlap on the GPU
@@ -438,13 +440,15 @@ fp8q_status fp8q_convert_e4m3(const float *in, uint8_t *out, size_t count, void 
 
 /*
  * Exhaustive device check of the quantizers' division. The quantizers form
- * x / s from the correctly rounded reciprocal of s and one remainder
- * correction instead of a full IEEE division per element. This call runs,
- * for every finite non-negative bf16 amax (s = max(amax, 1e-10f)/448) and
- * every bf16 x with |x| <= amax (both signs), that division and the IEEE
- * division, and compares the e4m3 codes and the fp32 quotients.
- *   counts  device pointer to 3 uint64: [0] pairs checked (1065402240),
- *           [1] code mismatches, [2] fp32 quotient mismatches.
+ * the scale s = max(amax, 1e-10f)/448 and its reciprocal with a remainder
+ * correction each, and x / s from that reciprocal and one more remainder
+ * correction, instead of IEEE divisions. This call runs, for every finite
+ * non-negative bf16 amax and every bf16 x with |x| <= amax (both signs),
+ * those steps and the IEEE ones, and compares the scales, reciprocals, e4m3
+ * codes and fp32 quotients.
+ *   counts  device pointer to 4 uint64: [0] pairs checked (1065402240),
+ *           [1] code mismatches, [2] fp32 quotient mismatches, [3] amax
+ *           values whose scale or reciprocal differs from the IEEE one.
  * Errors: NULL, UNSUPPORTED_DEVICE, CUDA.
  */
 fp8q_status fp8q_check_division(unsigned long long *counts, void *stream);
@@ -464,13 +468,32 @@ fp8q_status fp8q_check_division(unsigned long long *counts, void *stream);
  */
 fp8q_status fp8q_check_silu_mul(unsigned long long *counts, uint32_t *max_err_bits, void *stream);
 
+/*
+ * Diagnostic of the bounded waits (not part of the method): runs the two
+ * kernels of fp8q_linear on the same arguments (the multi-group quantizer,
+ * forced, then the GEMM that m selects) with every copy of their producers
+ * suppressed and every wait bounded by `wait_budget_cycles` SM clocks, so
+ * that each kernel's waits run out. Each kernel then raises its bit in the
+ * device error word (fp8q_device_error: bit 2 the quantizer, bit 0 the GEMM),
+ * lets nothing in flight outlive it, frees its tensor memory and returns; y
+ * and the workspace are left unspecified. The call returns FP8Q_OK once both
+ * kernels are enqueued; the context stays usable afterwards.
+ * wait_budget_cycles: 1 .. 2e9 (about one second at B200 clocks; tests pass
+ * about a millisecond). Errors: ARG, and those of fp8q_linear.
+ */
+fp8q_status fp8q_diag_stalled_linear(const void *x, const void *wq, const float *w_scale, void *y,
+                                     void *workspace, size_t workspace_bytes,
+                                     uint32_t m, uint32_t n, uint32_t k,
+                                     uint64_t wait_budget_cycles, void *stream);
+
 /* Number of kernels this library has launched in this process. */
 uint64_t fp8q_launch_count(void);
 
 /*
  * Read and clear the device error words of the current device: non-zero when
  * a kernel's bounded wait ran out (the kernel then stopped early and its
- * outputs are incomplete). Bit 0: an FP8 GEMM; bit 1: the NVFP4 GEMM. Synchronizes `stream` first. Returns FP8Q_OK or
+ * outputs are incomplete). Bit 0: an FP8 GEMM; bit 1: the NVFP4 GEMM; bit 2:
+ * the multi-group activation quantizer. Synchronizes `stream` first. Returns FP8Q_OK or
  * FP8Q_ERR_DEVICE_TIMEOUT (with *code set), or FP8Q_ERR_CUDA.
  */
 fp8q_status fp8q_device_error(void *stream, uint32_t *code);

@@ -161,8 +161,9 @@ def test_convert_matches_oracle_encoder_exhaustively():
 def test_division_exhaustive_against_ieee():
     """The quantizers' reciprocal-plus-correction division gives the code of the
     IEEE quotient for every (x, amax) pair of bf16 values with |x| <= amax."""
-    pairs, code_bad, quot_bad = api.check_division()
+    pairs, code_bad, quot_bad, scale_bad = api.check_division()
     assert pairs == 0x7F80 * 0x7F81
+    assert scale_bad == 0, "a group scale or its reciprocal differs from IEEE division"
     assert code_bad == 0
     print(f"division check: {pairs} pairs, {code_bad} code mismatches, {quot_bad} quotient mismatches")
 

@@ -115,22 +115,28 @@ def test_b200_floor_picks_the_faster_variant_at_decode_widths():
         assert p.variant == (api.MULTI if faster == "multi" else api.SINGLE), (m, k)
 
 
+FLOOR_CTAS_148 = 67  # ceil(0.45 * 148)
+
+
 def test_pick_keeps_kernel_and_grid_together():
+    # MULTI is the streaming kernel: one CTA per 16-group chunk, at most 3 per SM.
     for m in [1, 16, 17, 25, 53, 60, 100, 1168, 4576]:
         for k in [512, 5120, 6144, 17408]:
             auto = api.quant_pick(m, k, 148)
             g = k // 128
-            min_m = api.quant_floor_min_m(k, 148, 8, 4, 2.0 / 3.0)
-            assert auto.variant == (api.MULTI if m >= min_m else api.SINGLE)
+            chunks = -(-(m * g) // 16)
+            grid = min(chunks, 3 * 148)
             assert auto.forced == 0
-            assert auto.floor_ctas == 99
-            assert auto.multi_ctas == -(-g // 8) * -(-m // 4)
+            assert auto.floor_ctas == FLOOR_CTAS_148
+            assert auto.multi_ctas == grid
+            assert auto.variant == (api.MULTI if grid >= FLOOR_CTAS_148 else api.SINGLE)
             single = api.quant_pick(m, k, 148, api.SINGLE)
             assert single.variant == api.SINGLE and single.forced == 1
             assert single.grid_x == m * g and single.block_x == 16 and single.groups_per_cta == 1
             multi = api.quant_pick(m, k, 148, api.MULTI)
-            assert multi.variant == api.MULTI and multi.grid_x == multi.multi_ctas and multi.block_x == 64
-            assert multi.groups_per_cta == 32
+            assert multi.variant == api.MULTI and multi.grid_x == grid and multi.block_x == 224
+            assert multi.groups_per_cta == 16 * -(-chunks // grid)
+            assert multi.groups_per_cta * multi.grid_x >= m * g
 
 
 def test_pick_argument_errors():
