@@ -272,8 +272,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t r_local = quad * 32u + lane;
         const uint32_t tempty_even[2] = {mapa_shared(smem_addr(&sm.tempty[0]), 0),
                                          mapa_shared(smem_addr(&sm.tempty[1]), 0)};
-        // The activation scales come from the quantizer's K-major output.
-        if (kDirect) grid_dependency_wait();
+        // The activation scales come from the quantizer's K-major output,
+        // and nothing else in global memory is touched before the grid this
+        // launch depends on has completed either.
+        grid_dependency_wait();
         uint32_t it = 0;
         bool ok = true;
         for (uint32_t tile = pair; ok && tile < sh.num_tiles; tile += num_pairs) {

@@ -44,14 +44,16 @@ __global__ void __launch_bounds__(16) quant_act_single_kernel(const uint16_t* __
                                                              uint8_t* __restrict__ q, float* __restrict__ s_row,
                                                              float* __restrict__ s_k, uint32_t m, uint32_t k,
                                                              uint32_t mp) {
-    if (gridDim.x <= kSingleTriggerMaxGrid) trigger_dependents();
     const uint32_t G = k >> 7;
     const uint32_t t = blockIdx.x / G, g = blockIdx.x - t * G;
     const uint32_t lane = threadIdx.x;
     const size_t off = static_cast<size_t>(t) * k + static_cast<size_t>(g) * 128 + lane * 8;
     // Nothing is read or written in global memory before the grid this
-    // launch may depend on has completed.
+    // launch may depend on has completed; only then may the dependent (the
+    // GEMM of a fused linear) launch, so that everything before this kernel
+    // in the stream has completed when it starts.
     grid_dependency_wait();
+    if (gridDim.x <= kSingleTriggerMaxGrid) trigger_dependents();
     const uint4 v = ld_stream16(x + off);
     float f[8];
     widen8(v, f);
@@ -108,16 +110,17 @@ __global__ void __launch_bounds__(kStreamThreads, kStreamCtasPerSm)
     const uint32_t stride = gridDim.x * kStreamWarps;
     const uint32_t mine = first < chunks ? (chunks - 1 - first) / stride + 1 : 0;
 
-    // Let the dependent (the GEMM of a fused linear) launch early.
-    trigger_dependents();
     if (lane == 0) {
         for (uint32_t i = 0; i < kStreamSlots; ++i) mbar_init(&full[i], 1);
         fence_mbar_init();
     }
     __syncwarp();
     // Nothing is read or written in global memory before the grid this
-    // launch may depend on has completed.
+    // launch may depend on has completed; only then may the dependent (the
+    // GEMM of a fused linear) launch, so that everything before this kernel
+    // in the stream has completed when it starts.
     grid_dependency_wait();
+    trigger_dependents();
     zero_kmajor_pad(s_k, m, mp, G);
 
     auto issue = [&](uint32_t i) {
