@@ -377,6 +377,11 @@ def kernel_timings(wl: dict, dev, sms: int, hbm: float, fp8_peak: float, steps: 
     st, gr = both(lambda i: api.linear(sets[i % ns]["x"], sets[i % ns]["wq"], sets[i % ns]["ws"],
                                        workspace=sets[i % ns]["work"], out=sets[i % ns]["y"]), ns)
     out["linear"] = {"us_graph": gr, "us_stream": st, "tflops_graph": flops / (gr * 1e-6) / 1e12}
+    if m <= 32:
+        # The one-launch decode path (the GEMM quantizes x itself) beside it.
+        st, gr = both(lambda i: api.linear_decode_fused(sets[i % ns]["x"], sets[i % ns]["wq"], sets[i % ns]["ws"],
+                                                        workspace=sets[i % ns]["work"], out=sets[i % ns]["y"]), ns)
+        out["linear_decode_fused"] = {"us_graph": gr, "us_stream": st}
     out["rotation"] = {"quantizer_sets": nq, "gemm_sets": ns}
     del sets
     torch.cuda.empty_cache()
@@ -410,6 +415,90 @@ def decode_quant_arms(dev, sms: int, warmup: int) -> list:
             row["faster"] = "multi" if row["multi_us"] < row["single_us"] else "single"
             rows.append(row)
     return rows
+
+
+def nvfp4_hbm_bytes(m: int, n: int, k: int) -> int:
+    """Algorithmic bytes of one NVFP4 GEMM: both packed operands (half a byte
+    an element), their MMA-layout scales (one byte per 16 elements, rows
+    padded to 128) and the bf16 output."""
+    pad = lambda r: -(-r // 128) * 128
+    return m * k // 2 + n * k // 2 + (pad(m) + pad(n)) * k // 16 + 2 * m * n
+
+
+def nvfp4_pack_bytes(m: int, k: int) -> int:
+    """Algorithmic bytes of packing an [m, k] activation for the GEMM: read
+    bf16, write the packed E2M1 pairs and the MMA-layout scales."""
+    return 2 * m * k + m * k // 2 + (-(-m // 128) * 128) * k // 16
+
+
+def nvfp4_timings(m: int, n: int, k: int, dev, hbm: float, fp4_peak: float, steps: int, warmup: int) -> dict:
+    """The NVFP4 projection arm at one shape: the packer, the block-scaled FP4
+    GEMM and the fused projection (packer + GEMM), each in its own loop over
+    rotating inputs larger than L2, timed in CUDA graphs and on the stream.
+    The weight is a synthetic bf16 N(0, 0.02) packed with its global scale."""
+    import torch
+    from fp8_block_scaled_group_b200 import api
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(9000 + m + k)
+    reps = max(steps, 20)
+
+    def both(fn, nsets):
+        for i in range(max(warmup, nsets)):
+            fn(i)
+        torch.cuda.synchronize()
+        return stream_loop_ms(fn, max(reps, 2 * nsets)) * 1e3, graph_loop_ms(fn, max(reps, 2 * nsets)) * 1e3
+
+    gb = nvfp4_hbm_bytes(m, n, k)
+    ns = rotation(gb + 2 * m * k)
+    x0 = device_activations(m, k, 0.01, 20.0, gen, dev)
+    sets = []
+    for _ in range(ns):
+        w = (torch.randn((n, k), generator=gen, device=dev, dtype=torch.float32) * 0.02).to(torch.bfloat16)
+        s2w = float(w.float().abs().max().item()) / (6.0 * 448.0)
+        qw, _, sfw = api.nvfp4_quant(w, s2w, row_major=False)
+        del w
+        qa, _, sfa = api.nvfp4_quant(x0, 1.0, row_major=False)
+        sets.append(dict(x=x0.clone(), qa=qa, sfa=sfa, qw=qw, sfw=sfw, s2w=s2w,
+                         work=torch.empty(api.nvfp4_linear_workspace_bytes(m, k), dtype=torch.uint8, device=dev),
+                         y=torch.empty((m, n), dtype=torch.bfloat16, device=dev)))
+    out = {"m": m, "n": n, "k": k}
+    st, gr = both(lambda i: api.nvfp4_gemm(sets[i % ns]["qa"], sets[i % ns]["sfa"], 1.0, sets[i % ns]["qw"],
+                                           sets[i % ns]["sfw"], sets[i % ns]["s2w"], out=sets[i % ns]["y"]), ns)
+    flops = 2.0 * m * n * k
+    if m <= 64:
+        gm = {"bound": "hbm", "unit": "GB/s", "peak": hbm, "achieved": gb / (gr * 1e-6) / 1e9}
+    else:
+        gm = {"bound": "tensor", "unit": "TFLOP/s", "peak": fp4_peak, "achieved": flops / (gr * 1e-6) / 1e12,
+              "peak_source": "measured bf16 burst x 4 (fp4:bf16 nominal ratio; an assumption, FP4 is not measured)"}
+    gm.update(kernel="nvfp4_gemm_kernel", frac=gm["achieved"] / gm["peak"], us_graph=gr, us_stream=st,
+              algorithmic_bytes=gb, tflops=flops / (gr * 1e-6) / 1e12)
+    out["gemm"] = gm
+    pb = nvfp4_pack_bytes(m, k)
+    nq = rotation(pb)
+    xs = [x0.clone() for _ in range(nq)]
+    po = [(torch.empty((m, k // 2), dtype=torch.uint8, device=dev),
+           torch.empty((api.nvfp4_sf_mma_bytes(m, k),), dtype=torch.uint8, device=dev)) for _ in range(nq)]
+    import ctypes
+    from fp8_block_scaled_group_b200 import _lib
+    lib = _lib.load()
+
+    def pack(i):
+        q, sf = po[i % nq]
+        lib.fp8q_nvfp4_quant(ctypes.c_void_p(xs[i % nq].data_ptr()), ctypes.c_void_p(q.data_ptr()), None,
+                             ctypes.c_void_p(sf.data_ptr()), 1.0, m, k,
+                             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+    st, gr = both(pack, nq)
+    out["pack"] = {"bound": "hbm", "kernel": "nvfp4_quant_kernel", "bytes": pb, "us_graph": gr, "us_stream": st,
+                   "achieved": pb / (gr * 1e-6) / 1e9, "peak": hbm, "unit": "GB/s",
+                   "frac": pb / (gr * 1e-6) / 1e9 / hbm}
+    st, gr = both(lambda i: api.nvfp4_linear(sets[i % ns]["x"], sets[i % ns]["qw"], sets[i % ns]["sfw"],
+                                             sets[i % ns]["s2w"], workspace=sets[i % ns]["work"],
+                                             out=sets[i % ns]["y"]), ns)
+    out["linear"] = {"us_graph": gr, "us_stream": st, "tflops_graph": flops / (gr * 1e-6) / 1e12}
+    del sets, xs, po
+    torch.cuda.empty_cache()
+    return out
 
 
 # The configurations besides the headline one, timed kernel by kernel:
@@ -592,6 +681,11 @@ def ours_arm(args):
             if name != args.workload:
                 per_config[name] = kernel_timings(WORKLOADS[name], dev, sms, hbm, fp8_peak, args.steps, args.warmup)
         per_config["act_quant_decode_arms"] = decode_quant_arms(dev, sms, args.warmup)
+        fp4_peak = bf16 * 4.0  # fp4 dense = 4x bf16 dense (nominal 9 / 2.25 PF), an assumption
+        per_config["nvfp4_prefill_m1168_n17408_k5120"] = nvfp4_timings(1168, 17408, 5120, dev, hbm, fp4_peak,
+                                                                      args.steps, args.warmup)
+        per_config["nvfp4_decode_m25_n6144_k5120"] = nvfp4_timings(25, 6144, 5120, dev, hbm, fp4_peak,
+                                                                  args.steps, args.warmup)
     clk = clocks.stop()
 
     # End to end through the public call with host buffers: pinned X in,

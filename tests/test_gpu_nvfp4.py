@@ -3,10 +3,6 @@
 Packed E2M1 bytes and E4M3 scales (both layouts) and the FP8-to-bf16
 dequantizer: bit-exact. NVFP4 GEMM outputs: every compared element within
 |y - ref| <= 8e-3 |ref| + 1e-3 rms(ref) of the float64 reference.
-
-Pending: the NVFP4 kernels have not yet run on a GPU, so this file's name
-keeps it out of the collected suite. It becomes tests/test_gpu_nvfp4.py
-after its first run on a B200 (pytest tests/pending_gpu_nvfp4.py -m gpu).
 """
 import numpy as np
 import pytest
