@@ -48,6 +48,13 @@ FFN_WORKLOADS = {
     "ffn_m25_d5120_i17408": dict(m=25, d=5120, i=17408, seed=1100),
 }
 FFN_METRIC = "dense FFN (FP8 block-scaled, x quantized once) TFLOP/s"
+# The NVFP4 projection arm at the FP8 path's shapes (x packed to E2M1 with
+# E4M3 block scales inside the call, times a packed weight).
+NVFP4_WORKLOADS = {
+    "nvfp4_m1168_n17408_k5120": dict(m=1168, n=17408, k=5120, seed=1200),
+    "nvfp4_m25_n6144_k5120": dict(m=25, n=6144, k=5120, seed=1201),
+}
+NVFP4_METRIC = "NVFP4 projection (x packed in the call) TFLOP/s"
 DEFAULT_WORKLOAD = "prefill_m1168_n17408_k5120"
 N_SETS = 3
 
@@ -82,8 +89,8 @@ def gemm_hbm_bytes(m, n, k):
 KERNEL_SOURCES = {
     "gemm_blockscaled_kernel": ["gemm.cu", "group_quant.cuh", "ptx.cuh", "internal.h"],
     "gemm_decode_kernel": ["gemm.cu", "group_quant.cuh", "ptx.cuh", "internal.h"],
-    "quant_act_multi_kernel": ["quant.cu", "group_quant.cuh", "ptx.cuh"],
-    "quant_act_single_kernel": ["quant.cu", "group_quant.cuh", "ptx.cuh"],
+    "quant_act_stream_kernel": ["quant.cu", "group_quant.cuh", "ptx.cuh", "internal.h"],
+    "quant_act_single_kernel": ["quant.cu", "group_quant.cuh", "ptx.cuh", "internal.h"],
     "silu_mul_quant_kernel": ["ffn.cu", "group_quant.cuh", "ptx.cuh"],
 }
 
@@ -501,6 +508,41 @@ def nvfp4_timings(m: int, n: int, k: int, dev, hbm: float, fp4_peak: float, step
     return out
 
 
+def quant_variant_sweep(dev, sms: int) -> list:
+    """Both activation-quantizer variants, forced, over M x K (CUDA graphs
+    of back-to-back launches over rotating inputs larger than 3x L2): the
+    measurements the SINGLE/MULTI floor is derived from."""
+    import torch
+    from fp8_block_scaled_group_b200 import api
+    rows = []
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4242)
+    for k in (5120, 6144, 17408):
+        for m in (1, 4, 8, 16, 17, 20, 24, 25, 32, 40, 48, 56, 64, 80, 96, 128, 256, 512, 1168, 4576):
+            g, mp = k // 128, api.m_pad(m)
+            nq = rotation(quant_bytes(m, k), hi=64)
+            base = [device_activations(m, k, 0.01, 20.0, gen, dev) for _ in range(min(nq, 2))]
+            xs = [base[i % len(base)] if i < len(base) else base[i % len(base)].clone() for i in range(nq)]
+            qo = [(torch.empty((m, k), dtype=torch.uint8, device=dev), torch.empty((m, g), dtype=torch.float32, device=dev),
+                   torch.empty((g, mp), dtype=torch.float32, device=dev)) for _ in range(nq)]
+            row = {"m": m, "k": k}
+            for name, var in (("single", api.SINGLE), ("multi", api.MULTI)):
+                fn = lambda i, var=var: api.quant_act(xs[i % nq], variant=var, out=qo[i % nq])
+                for i in range(nq):
+                    fn(i)
+                torch.cuda.synchronize()
+                row[name + "_us"] = graph_loop_ms(fn, max(64, 2 * nq)) * 1e3
+            pick = api.quant_pick(m, k, sms)
+            row["multi_ctas"] = pick.multi_ctas
+            row["picked"] = "multi" if pick.variant == api.MULTI else "single"
+            row["faster"] = "multi" if row["multi_us"] < row["single_us"] else "single"
+            rows.append(row)
+            print(json.dumps(row), flush=True)
+            del xs, qo, base
+            torch.cuda.empty_cache()
+    return rows
+
+
 # The configurations besides the headline one, timed kernel by kernel:
 # decode widths at both K and the M=4576 prefill at both K.
 PER_CONFIG = ["decode_m25_n6144_k5120", "decode_m25_n5120_k17408",
@@ -526,6 +568,13 @@ def grow_sample(run, m: int, threads: int, target_s: float):
         rows = grown
         t = run(rows)
     return rows, t
+
+
+def sample_kind(rows: int, m: int) -> str:
+    """How a reference arm's ms_per_step was obtained from its timed rows."""
+    if rows >= m:
+        return f"measured: each step times all {m} token rows"
+    return f"extrapolated: each step times {rows} of {m} token rows and scales that time to the whole step"
 
 
 def cpu_oracle_sample(wl: dict, seed: int, target_s: float, threads: int, per_row: bool = False,
@@ -587,8 +636,7 @@ def reference_arm(args):
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": flops / (value * 1e12) * 1e3,
-        "ms_per_step_kind": f"extrapolated: each step times {rows} of {wl['m']} token rows and scales that "
-                            f"time to the whole step",
+        "ms_per_step_kind": sample_kind(rows, wl["m"]),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "m": wl["m"], "n": wl["n"], "k": wl["k"]},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
@@ -833,8 +881,7 @@ def ffn_reference_arm(args):
         "impl": "reference", "metric": FFN_METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": flops / (value * 1e12) * 1e3, "higher_is_better": True, "scaling": "weak",
-        "ms_per_step_kind": f"extrapolated: each step times {rows} of {m} token rows and scales that time "
-                            f"to the whole step",
+        "ms_per_step_kind": sample_kind(rows, m),
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "m": m, "d": d, "i": i},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
@@ -980,13 +1027,162 @@ def ffn_arm(args):
     return 0
 
 
+def nvfp4_oracle_sample(wl: dict, threads: int, target_s: float, rows: int | None = None):
+    """The oracle's NVFP4 projection on a bounded sample of token rows:
+    pack those rows of x, then their float64 reference rows. Weight packing
+    is not part of the step and is done once. Returns (TFLOP/s, rows, s)."""
+    import oracle
+    from fp8_block_scaled_group_b200 import inputs
+    m, n, k = wl["m"], wl["n"], wl["k"]
+    xb = inputs.activations(m, k, wl["seed"])
+    key = ("nvfp4", n, k, wl["seed"])
+    if key not in _FFN_ORACLE_W:
+        wb = inputs.weights(n, k, wl["seed"] + 1)
+        s2w = oracle.nvfp4_global_scale(wb)
+        _FFN_ORACLE_W[key] = (*oracle.nvfp4_quant(wb, s2w), s2w)
+    qw, sfw, s2w = _FFN_ORACLE_W[key]
+
+    def run(r):
+        t0 = time.perf_counter()
+        qa, sfa = oracle.nvfp4_quant(np.ascontiguousarray(xb[:r]), 1.0)
+        oracle.nvfp4_gemm_ref(qa, sfa, 1.0, qw, sfw, s2w)
+        return time.perf_counter() - t0
+
+    if rows is None:
+        rows, t = grow_sample(run, m, threads, target_s)
+    else:
+        t = run(rows)
+    return 2.0 * rows * n * k / t / 1e12, rows, t
+
+
+def nvfp4_reference_arm(args):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    wl = NVFP4_WORKLOADS[args.workload]
+    threads = os.cpu_count() or 1
+    per_step = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    vals, rows = [], None
+    for j in range(args.warmup + args.steps):
+        v, rows, _ = nvfp4_oracle_sample(wl, threads, per_step, rows=rows)
+        if j >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals)
+    m, n, k = wl["m"], wl["n"], wl["k"]
+    print(json.dumps({
+        "impl": "reference", "metric": NVFP4_METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 2.0 * m * n * k / (value * 1e12) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step_kind": sample_kind(rows, m),
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "m": m, "n": n, "k": k},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{rows} of {m} token rows per step, scaled to the metric's unit"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+    return 0
+
+
+def nvfp4_arm(args):
+    """One step = one fp8q_nvfp4_linear call: pack x (E2M1 + E4M3 block
+    scales) and the block-scaled FP4 GEMM against a packed weight."""
+    import torch
+    from fp8_block_scaled_group_b200 import api, inputs
+
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = NVFP4_WORKLOADS[args.workload]
+    m, n, k = wl["m"], wl["n"], wl["k"]
+    to_dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).to(dev)
+    sets = []
+    for j in range(N_SETS):
+        xb = inputs.activations(m, k, rank_input_seed(wl["seed"], rank, j))
+        w = to_dev(inputs.weights(n, k, wl["seed"] + 1 + j))
+        s2w = float(w.float().abs().max().item()) / (6.0 * 448.0)
+        qw, _, sfw = api.nvfp4_quant(w, s2w, row_major=False)
+        del w
+        sets.append(dict(x=to_dev(xb), xb=xb, qw=qw, sfw=sfw, s2w=s2w,
+                         work=torch.empty(api.nvfp4_linear_workspace_bytes(m, k), dtype=torch.uint8, device=dev),
+                         y=torch.empty((m, n), dtype=torch.bfloat16, device=dev)))
+    n_sets = rotation(n * k // 2 + 3 * m * k + 2 * m * n, lo=N_SETS)
+    for j in range(N_SETS, n_sets):
+        b = sets[j % N_SETS]
+        sets.append(dict(b, x=b["x"].clone(), qw=b["qw"].clone(), sfw=b["sfw"].clone(),
+                         work=torch.empty_like(b["work"]), y=torch.empty_like(b["y"])))
+    torch.cuda.synchronize()
+
+    def step(j):
+        s = sets[j % n_sets]
+        api.nvfp4_linear(s["x"], s["qw"], s["sfw"], s["s2w"], workspace=s["work"], out=s["y"])
+
+    for j in range(args.warmup):
+        step(j)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    l0 = api.launch_count()
+    ms = max_over_ranks(stream_loop_ms(step, args.steps), world)
+    launches = api.launch_count() - l0
+    hbm, bf16, _, src = load_peaks()
+    kt = nvfp4_timings(m, n, k, dev, hbm, bf16 * 4.0, args.steps, args.warmup)
+    clk = clocks.stop()
+    x_host = [torch.from_numpy(s["xb"].view(np.int16)).view(torch.bfloat16).pin_memory() for s in sets[:N_SETS]]
+    y_host = torch.empty((m, n), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty((m, k), dtype=torch.bfloat16, device=dev)
+
+    def e2e(j):
+        s = sets[j % n_sets]
+        x_dev.copy_(x_host[j % N_SETS], non_blocking=True)
+        api.nvfp4_linear(x_dev, s["qw"], s["sfw"], s["s2w"], workspace=s["work"], out=s["y"])
+        y_host.copy_(s["y"], non_blocking=True)
+
+    for j in range(args.warmup):
+        e2e(j)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(stream_loop_ms(e2e, args.steps), world)
+    flops = 2.0 * m * n * k
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        v, rows, t = nvfp4_oracle_sample(wl, threads, args.cpu_seconds)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{rows} of {m} token rows of one step (pack + float64 reference rows), {t:.1f} s"}
+    if rank == 0:
+        gm = kt["gemm"]
+        print(json.dumps({
+            "metric": NVFP4_METRIC, "value": weak_scaling_value(flops, world, 1, ms) / 1e12, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e2m1", "data": "synthetic",
+            "config": {"workload": args.workload, "m": m, "n": n, "k": k, "parallelism": f"replicas{world}",
+                       "l2": f"{n_sets} rotating input sets for the step; kernel loops rotate > 3x L2"},
+            "roofline": {"bound": gm["bound"], "kernel": gm["kernel"], "achieved": gm["achieved"], "peak": gm["peak"],
+                         "unit": gm["unit"], "frac": gm["frac"], "traffic": None, "us": gm["us_graph"],
+                         "us_stream_loop": gm["us_stream"], "algorithmic_bytes": gm["algorithmic_bytes"],
+                         "peak_source": gm.get("peak_source", f"{src} copy bandwidth")},
+            "pack": kt["pack"], "linear_us": kt["linear"],
+            "cpu_baseline": cpu,
+            "e2e": {"value": weak_scaling_value(flops, world, 1, e2e_ms) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": m * k * 2, "d2h_bytes_per_step": m * n * 2},
+            "gpu_launches": int(sum_over_ranks(launches, world)),
+            "clocks": clk,
+        }), flush=True)
+    barrier(world)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(FFN_WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(FFN_WORKLOADS) + sorted(NVFP4_WORKLOADS),
+                    default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
@@ -995,6 +1191,8 @@ def main():
                     help="weight scales per 128x128 block (the pages' format) or one per weight row")
     ap.add_argument("--decode-path", choices=["two_launch", "fused"], default="two_launch",
                     help="decode widths (M <= 32): quantizer + GEMM, or the GEMM with the quantizer fused in")
+    ap.add_argument("--quant-sweep", action="store_true",
+                    help="time both quantizer variants over M x K on cuda:0 (one JSON row each) and exit")
     ap.add_argument("--kernel-digests", action="store_true",
                     help="print the source digest of each kernel (the key of profiles/traffic.txt) and exit")
     args = ap.parse_args()
@@ -1002,11 +1200,20 @@ def main():
         for kname in KERNEL_SOURCES:
             print(kname, kernel_digest(kname))
         return 0
+    if args.quant_sweep:
+        import torch
+        dev = torch.device("cuda", 0)
+        quant_variant_sweep(dev, torch.cuda.get_device_properties(dev).multi_processor_count)
+        return 0
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
     if args.workload in FFN_WORKLOADS:
         if args.impl == "reference":
             return ffn_reference_arm(args)
         return ffn_arm(args)
+    if args.workload in NVFP4_WORKLOADS:
+        if args.impl == "reference":
+            return nvfp4_reference_arm(args)
+        return nvfp4_arm(args)
     if args.impl == "reference":
         return reference_arm(args)
     return ours_arm(args)

@@ -22,9 +22,9 @@ constexpr uint32_t kStreamCtasPerSm = 3;
 // MULTI runs when its grid (one CTA per chunk, at most kStreamCtasPerSm per
 // SM) holds at least this many CTAs per SM; below it the one-group-per-CTA
 // kernel's many small CTAs finish sooner. From a B200 sweep of both variants
-// over M in 1..4576 at K = 5120, 6144, 17408: SINGLE was faster up to 63
-// MULTI CTAs and MULTI from 68 on, so the floor is ceil(0.45 * 148) = 67.
-constexpr float kMultiMinCtasPerSm = 0.45f;
+// over M in 1..4576 at K = 5120, 6144, 17408: SINGLE was faster up to 68
+// MULTI CTAs and MULTI from 72 on, so the floor is ceil(0.47 * 148) = 70.
+constexpr float kMultiMinCtasPerSm = 0.47f;
 
 // CTAs of the MULTI grid for (m, k) on `sms` SMs.
 uint32_t stream_grid(uint32_t m, uint32_t k, uint32_t sms);
