@@ -42,7 +42,6 @@
 #include <cudaTypedefs.h>
 
 #include <cstdlib>
-#include <cstring>
 #include <mutex>
 
 #include "group_quant.cuh"
@@ -398,355 +397,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 for (uint32_t it = first; it < issued; ++it)
                     mbar_wait(&sm.sfull[it % kScaleStages], (it / kScaleStages) & 1u, &never);
             }
-            spin_cycles(200000);
-        }
-        __syncthreads();
-    }
-    cluster_sync_all();  // no remote arrive or pair MMA can still target this CTA
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc_pair(tmem, kTmemCols);
-    }
-}
-
-// ------------------------------------------ prefill with swapped operands --
-//
-// The same contraction with the weight on the MMA's M and the tokens on its
-// N: a CTA pair owns 256 weight rows (128 in each CTA's TMEM lanes) and a
-// tile of up to 256 tokens (TMEM columns). The tile's token count is
-// ceil16(M - t0), so a ragged last token tile costs MMA time in proportion
-// to its tokens (N is any multiple of 16), where the token-on-M kernel pays
-// for a full 256-row tile. At M = 1168 (4 x 256 + 144) that removes the
-// 8.75 % of the MMA work spent on zero rows, and with tiles visited
-// token-fastest every pair that runs five tiles runs exactly one short one.
-//
-//   D[n][j] = sum_k wq[n][k] * q[t0 + j][k]                (tcgen05, fp32, TMEM)
-//   acc[n][j] += (w_s[n/128][g] * a_s[t0 + j][g]) * D[n][j]  (promotion)
-//
-// A CTA's 128 weight rows are one weight block, so the K block's scale is a
-// vector over the tile's columns, c[j] = w_s[n/128][g] * a_s[t0 + j][g]
-// (a_s alone for per-row weights, whose scale the epilogue applies per row):
-// warp 3 builds it from the K-major activation scales into a 4-slot
-// shared-memory ring and every promotion thread reads it (broadcast loads).
-// Warps 0-2 as in the token-on-M kernel (TMA producer, two MMA issuers);
-// warps 4-11 promote and store, warp w taking TMEM lanes 32*(w%4).. and one
-// of two column ranges of the tile, split at ceil16(Nt/2). The epilogue
-// writes y[t][n] for its 32 rows n: one instruction stores 32 consecutive
-// bf16 of a token row.
-
-constexpr uint32_t kSwSlots = 4;  // column-scale vectors in flight
-
-struct __align__(1024) SwapSmem {
-    uint8_t w[kStages][BM * BK];      // this CTA's 128 weight rows of a K block
-    uint8_t t[kStages][BN_CTA * BK];  // this CTA's half of the token tile (128 rows staged)
-    float ascale[kSwSlots][BN];       // a_s[t0 .. t0+255][g], copied by TMA
-    float colscale[kSwSlots][BN];     // c[j] = w_s[n/128][g] * a_s[t0 + j][g]
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
-    uint64_t sfull[kSwSlots];
-    uint64_t sempty[kSwSlots];
-    uint64_t cfull[kSwSlots];
-    uint64_t cempty[kSwSlots];
-    uint64_t tfull[2];
-    uint64_t tempty[2];
-    uint64_t mma_done[2];
-    uint32_t tmem_base;
-    uint32_t abort;
-    uint32_t consumed[2];
-};
-
-constexpr size_t kSwapSmemBytes = sizeof(SwapSmem) + 1024;
-
-struct SwapShape {
-    uint32_t M, N, G, Mp;
-    uint32_t num_t, num_tiles;  // token tiles, tiles
-    uint32_t w_per_row;
-    uint32_t no_copies;
-    long long budget;
-};
-
-// Token tile tt of a tile: tokens t0 .. t0 + nt - 1 (nt a multiple of 16,
-// at most 256; rows past M are zero in the operand and never stored).
-__device__ __forceinline__ void swap_coords(const SwapShape& sh, uint32_t tile, uint32_t& t0, uint32_t& nt,
-                                            uint32_t& n0) {
-    const uint32_t tt = tile % sh.num_t;
-    n0 = (tile / sh.num_t) * BM_PAIR;
-    t0 = tt * BN;
-    const uint32_t rest = sh.M - t0;
-    nt = rest >= BN ? BN : (rest + 15u) / 16u * 16u;
-}
-
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    gemm_swapped_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmT,
-                        const __grid_constant__ CUtensorMap tmS, const float* __restrict__ w_s,
-                        uint16_t* __restrict__ y, const SwapShape sh) {
-    extern __shared__ uint8_t smem_raw[];
-    SwapSmem& sm = *reinterpret_cast<SwapSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t warp = threadIdx.x >> 5;
-    const uint32_t lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_ctarank();
-    const uint32_t pair = blockIdx.x >> 1;
-    const uint32_t num_pairs = gridDim.x >> 1;
-    volatile uint32_t* abort = &sm.abort;
-
-    if (threadIdx.x == 0) {
-        for (uint32_t s = 0; s < kStages; ++s) {
-            mbar_init(&sm.full[s], 2);  // one expect-tx arrival from each CTA of the pair
-            mbar_init(&sm.empty[s], 1);
-        }
-        for (uint32_t c = 0; c < kSwSlots; ++c) {
-            mbar_init(&sm.sfull[c], 1);
-            mbar_init(&sm.sempty[c], 1);
-            mbar_init(&sm.cfull[c], 1);
-            mbar_init(&sm.cempty[c], kEpiWarps);
-        }
-        for (uint32_t b = 0; b < 2; ++b) {
-            mbar_init(&sm.tfull[b], 1);
-            mbar_init(&sm.tempty[b], 2 * kEpiWarps);  // promotion warps of both CTAs
-        }
-        mbar_init(&sm.mma_done[0], 1);
-        mbar_init(&sm.mma_done[1], 1);
-        sm.abort = 0;
-        sm.consumed[0] = sm.consumed[1] = 0;
-        fence_mbar_init();
-    }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmW);
-        tma_prefetch_desc(&tmT);
-        tma_prefetch_desc(&tmS);
-    }
-    if (warp == 1) {
-        tmem_alloc_pair(&sm.tmem_base, kTmemCols);
-        tmem_relinquish_pair();
-    }
-    tc_fence_before();
-    cluster_sync_all();  // barriers of both CTAs initialised before any remote arrive
-    tc_fence_after();
-    const uint32_t tmem = sm.tmem_base;
-    const uint32_t G = sh.G;
-    uint32_t issued = 0;
-
-    if (warp < 4) {
-        regs_dec<kRegsLow>();
-        if (warp == 0 && lane == 0 && !sh.no_copies) {
-            grid_dependency_wait();
-            uint32_t it = 0;
-            bool ok = true;
-            for (uint32_t tile = pair; ok && tile < sh.num_tiles; tile += num_pairs) {
-                uint32_t t0, nt, n0;
-                swap_coords(sh, tile, t0, nt, n0);
-                const int32_t my_w = static_cast<int32_t>(n0 + rank * BM);
-                const int32_t my_t = static_cast<int32_t>(t0 + rank * (nt / 2u));
-                for (uint32_t kb = 0; kb < G; ++kb, ++it) {
-                    const uint32_t s = it % kStages;
-                    const uint32_t ph = (it / kStages) & 1u;
-                    if (!mbar_wait(&sm.empty[s], ph ^ 1u, abort, sh.budget)) {
-                        ok = false;
-                        break;
-                    }
-                    // this CTA's copy of the K block's activation scales of the tile
-                    const uint32_t c = it % kSwSlots;
-                    if (!mbar_wait(&sm.sempty[c], ((it / kSwSlots) & 1u) ^ 1u, abort, sh.budget)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&sm.sfull[c], BN * 4u);
-                    tma_load_2d(sm.ascale[c], &tmS, &sm.sfull[c], static_cast<int32_t>(t0), static_cast<int32_t>(kb));
-                    const uint32_t full_even = mapa_shared(smem_addr(&sm.full[s]), 0);
-                    mbar_arrive_expect_tx_cluster(full_even, kTileBytesA + kTileBytesB);
-                    tma_load_2d_pair(sm.w[s], &tmW, full_even, static_cast<int32_t>(kb * BK), my_w);
-                    tma_load_2d_pair(sm.t[s], &tmT, full_even, static_cast<int32_t>(kb * BK), my_t);
-                    issued = it + 1;
-                }
-            }
-        } else if ((warp == 1 || warp == 2) && lane == 0 && rank == 0) {
-            // Two MMA issuers, one per TMEM buffer, as in the token-on-M kernel.
-            const uint32_t par = warp - 1u;
-            uint32_t it = 0;
-            bool ok = true;
-            for (uint32_t tile = pair; ok && tile < sh.num_tiles; tile += num_pairs) {
-                uint32_t t0, nt, n0;
-                swap_coords(sh, tile, t0, nt, n0);
-                const uint32_t idesc = idesc_e4m3_f32(BM_PAIR, nt);
-                for (uint32_t kb = 0; kb < G; ++kb, ++it) {
-                    if ((it & 1u) != par) continue;
-                    const uint32_t s = it % kStages;
-                    const uint32_t ph = (it / kStages) & 1u;
-                    const uint32_t b = it & 1u;
-                    const uint32_t tph = (it >> 1) & 1u;
-                    if (!mbar_wait(&sm.full[s], ph, abort, sh.budget)) {
-                        ok = false;
-                        break;
-                    }
-                    sm.consumed[par] = it + 1;
-                    if (!mbar_wait(&sm.tempty[b], tph ^ 1u, abort, sh.budget)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t d = tmem + b * BN;
-                    const uint64_t ad = smem_desc_k_sw128(smem_addr(sm.w[s]));
-                    const uint64_t bd = smem_desc_k_sw128(smem_addr(sm.t[s]));
-#pragma unroll
-                    for (uint32_t kk = 0; kk < BK / 32; ++kk)
-                        mma_f8f6f4_pair(d, ad + 2u * kk, bd + 2u * kk, idesc, kk > 0 ? 1u : 0u);
-                    mma_commit_pair_multicast(&sm.empty[s], 0x3);
-                    mma_commit_pair_multicast(&sm.tfull[b], 0x3);
-                }
-            }
-            mma_commit_pair(&sm.mma_done[par]);
-            volatile uint32_t never = 0;
-            mbar_wait(&sm.mma_done[par], 0, &never);
-        } else if (warp == 3 && !sh.no_copies) {
-            // Column scales of each K block of each tile, in both CTAs: the
-            // TMA-copied activation scales times this CTA's weight-block
-            // scale, eight columns a lane.
-            grid_dependency_wait();
-            uint32_t it = 0;
-            bool ok = true;
-            for (uint32_t tile = pair; ok && tile < sh.num_tiles; tile += num_pairs) {
-                uint32_t t0, nt, n0;
-                swap_coords(sh, tile, t0, nt, n0);
-                const uint32_t nb = (n0 + rank * BM) / BM;
-                const bool w_ok = n0 + rank * BM < sh.N;
-                const float* ws_row = w_s + static_cast<size_t>(w_ok && !sh.w_per_row ? nb : 0u) * G;
-                float w_next = sh.w_per_row ? 1.0f : __ldg(ws_row);
-                for (uint32_t kb = 0; kb < G; ++kb, ++it) {
-                    const uint32_t c = it % kSwSlots;
-                    const uint32_t cph = (it / kSwSlots) & 1u;
-                    const float wsc = w_next;
-                    if (!sh.w_per_row && kb + 1 < G) w_next = __ldg(ws_row + kb + 1);
-                    const bool got = mbar_wait(&sm.sfull[c], cph, abort, sh.budget) &&
-                                     mbar_wait(&sm.cempty[c], cph ^ 1u, abort, sh.budget);
-                    if (!__all_sync(0xFFFFFFFFu, got)) {
-                        ok = false;
-                        break;
-                    }
-                    const float4* a4 = reinterpret_cast<const float4*>(sm.ascale[c]);
-                    float4* c4 = reinterpret_cast<float4*>(sm.colscale[c]);
-                    const float4 u = a4[lane], v = a4[lane + 32];
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.sempty[c]);  // the copied scales are read
-                    c4[lane] = make_float4(wsc * u.x, wsc * u.y, wsc * u.z, wsc * u.w);
-                    c4[lane + 32] = make_float4(wsc * v.x, wsc * v.y, wsc * v.z, wsc * v.w);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.cfull[c]);
-                }
-            }
-        }
-    } else {
-        regs_inc<kRegsHigh>();
-        const uint32_t quad = warp & 3u;
-        const uint32_t half = (warp - 4u) >> 2;
-        const uint32_t lane_off = (quad * 32u) << 16;
-        const uint32_t tempty_even[2] = {mapa_shared(smem_addr(&sm.tempty[0]), 0),
-                                         mapa_shared(smem_addr(&sm.tempty[1]), 0)};
-        grid_dependency_wait();
-        uint32_t it = 0;
-        bool ok = true;
-        for (uint32_t tile = pair; ok && tile < sh.num_tiles; tile += num_pairs) {
-            uint32_t t0, nt, n0;
-            swap_coords(sh, tile, t0, nt, n0);
-            const uint32_t n = n0 + rank * BM + quad * 32u + lane;  // this thread's weight row
-            const uint32_t split = (nt / 2u + 15u) / 16u * 16u;
-            const uint32_t c0 = half ? split : 0u;                  // this warp's first column
-            const uint32_t ncols = half ? nt - split : split;       // a multiple of 16, at most 128
-            float2 acc[64];
-#pragma unroll
-            for (uint32_t i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
-            for (uint32_t kb = 0; kb < G; ++kb, ++it) {
-                const uint32_t b = it & 1u;
-                const uint32_t tph = (it >> 1) & 1u;
-                const uint32_t c = it % kSwSlots;
-                const uint32_t cph = (it / kSwSlots) & 1u;
-                const bool got = mbar_wait(&sm.cfull[c], cph, abort, sh.budget) &&
-                                 mbar_wait(&sm.tfull[b], tph, abort, sh.budget);
-                if (!__all_sync(0xFFFFFFFFu, got)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t taddr = tmem + lane_off + b * BN + c0;
-                const float4* cs = reinterpret_cast<const float4*>(&sm.colscale[c][c0]);
-#pragma unroll
-                for (uint32_t ch = 0; ch < 2; ++ch) {
-                    if (ch * 64u + 64u <= ncols) {
-                        uint32_t v[64];
-                        tmem_load64(taddr + ch * 64u, v);
-#pragma unroll
-                        for (uint32_t i = 0; i < 16; ++i) {
-                            const float4 s4 = cs[ch * 16u + i];
-                            acc[ch * 32 + 2 * i] = __ffma2_rn(
-                                make_float2(s4.x, s4.y),
-                                make_float2(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1])),
-                                acc[ch * 32 + 2 * i]);
-                            acc[ch * 32 + 2 * i + 1] = __ffma2_rn(
-                                make_float2(s4.z, s4.w),
-                                make_float2(__uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3])),
-                                acc[ch * 32 + 2 * i + 1]);
-                        }
-                    } else {
-#pragma unroll
-                        for (uint32_t q = 0; q < 4; ++q) {
-                            const uint32_t col = ch * 64u + q * 16u;
-                            if (col < ncols) {
-                                float v[16];
-                                tmem_load16(taddr + col, v);
-#pragma unroll
-                                for (uint32_t i = 0; i < 4; ++i) {
-                                    const float4 s4 = cs[col / 4u + i];
-                                    acc[col / 2u + 2 * i] = __ffma2_rn(make_float2(s4.x, s4.y),
-                                                                        make_float2(v[4 * i], v[4 * i + 1]),
-                                                                        acc[col / 2u + 2 * i]);
-                                    acc[col / 2u + 2 * i + 1] = __ffma2_rn(make_float2(s4.z, s4.w),
-                                                                            make_float2(v[4 * i + 2], v[4 * i + 3]),
-                                                                            acc[col / 2u + 2 * i + 1]);
-                                }
-                            }
-                        }
-                    }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive_cluster(tempty_even[b]);
-                    mbar_arrive(&sm.cempty[c]);
-                }
-            }
-            if (ok && n < sh.N) {
-                const float wr = sh.w_per_row ? __ldg(w_s + n) : 1.0f;
-                uint16_t* dst = y + static_cast<size_t>(t0 + c0) * sh.N + n;
-#pragma unroll
-                for (uint32_t i = 0; i < 64; ++i) {
-                    const uint32_t j = 2u * i;  // column within this warp's range
-                    if (j < ncols) {
-                        float2 a = acc[i];
-                        if (sh.w_per_row) a = __fmul2_rn(a, make_float2(wr, wr));
-                        const __nv_bfloat162 h = __floats2bfloat162_rn(a.x, a.y);
-                        if (t0 + c0 + j < sh.M) dst[static_cast<size_t>(j) * sh.N] = __bfloat16_as_ushort(h.x);
-                        if (t0 + c0 + j + 1 < sh.M) dst[static_cast<size_t>(j + 1) * sh.N] = __bfloat16_as_ushort(h.y);
-                    }
-                }
-            }
-        }
-    }
-
-    // Teardown, as in the token-on-M kernel; the scale copies this CTA
-    // started are waited for too.
-    tc_fence_before();
-    __syncthreads();
-    if (*abort) {
-        volatile uint32_t never = 0;
-        if (threadIdx.x == 0) atomicOr(&g_device_error, 1u);
-        if (warp == 0 && lane == 0) {
-            if (rank == 0) {
-                const uint32_t from = sm.consumed[0] < sm.consumed[1] ? sm.consumed[0] : sm.consumed[1];
-                for (uint32_t it = from; it < issued; ++it)
-                    if (it >= sm.consumed[it & 1u]) mbar_wait(&sm.full[it % kStages], (it / kStages) & 1u, &never);
-            }
-            const uint32_t first = issued > kSwSlots ? issued - kSwSlots : 0u;
-            for (uint32_t it = first; it < issued; ++it)
-                mbar_wait(&sm.sfull[it % kSwSlots], (it / kSwSlots) & 1u, &never);
             spin_cycles(200000);
         }
         __syncthreads();
@@ -1179,15 +829,6 @@ const KernelSetup& setup_for_device() {
             if (k.err == cudaSuccess && static_cast<uint32_t>(attr.numRegs) < kLaunchRegsNeeded)
                 k.err = cudaErrorInvalidConfiguration;
         }
-        if (k.err == cudaSuccess)
-            k.err = cudaFuncSetAttribute(gemm_swapped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSwapSmemBytes));
-        if (k.err == cudaSuccess) {
-            cudaFuncAttributes attr;
-            k.err = cudaFuncGetAttributes(&attr, gemm_swapped_kernel);
-            if (k.err == cudaSuccess && static_cast<uint32_t>(attr.numRegs) < kLaunchRegsNeeded)
-                k.err = cudaErrorInvalidConfiguration;
-        }
         if (k.err == cudaSuccess) k.err = cudaDeviceGetAttribute(&k.sms, cudaDevAttrMultiProcessorCount, dev);
     }
     return k;
@@ -1273,57 +914,6 @@ cudaError_t launch_decode(const GemmLaunch& L, int sms, cudaStream_t stream) {
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-// FP8Q_PREFILL=pair|swapped forces the prefill kernel (read once).
-int env_prefill() {
-    static const int v = [] {
-        const char* e = std::getenv("FP8Q_PREFILL");
-        if (!e) return 0;
-        if (!std::strcmp(e, "pair")) return 1;
-        if (!std::strcmp(e, "swapped")) return 2;
-        return 0;
-    }();
-    return v;
-}
-
-bool use_swapped(const GemmLaunch& L) {
-    const int forced = env_prefill();
-    if (forced) return forced == 2;
-    return false;
-}
-
-cudaError_t launch_swapped(const GemmLaunch& L, int sms, cudaStream_t stream) {
-    CUtensorMap tw, tt, ts;
-    if (!make_map_u8(&tw, L.wq, L.k, L.n, BM) || !make_map_u8(&tt, L.q, L.k, L.m, BN_CTA) ||
-        !make_map_scales_box(&ts, L.s_k, L.mp, L.k / BK, BN))
-        return cudaErrorInvalidValue;
-    SwapShape sh;
-    sh.M = L.m;
-    sh.N = L.n;
-    sh.G = L.k / BK;
-    sh.Mp = L.mp;
-    sh.num_t = (L.m + BN - 1) / BN;
-    sh.num_tiles = sh.num_t * ((L.n + BM_PAIR - 1) / BM_PAIR);
-    sh.w_per_row = L.w_per_row ? 1u : 0u;
-    sh.no_copies = L.diag_budget != 0 ? 1u : 0u;
-    sh.budget = L.diag_budget != 0 ? L.diag_budget : kWaitBudgetCycles;
-    const uint32_t max_pairs = static_cast<uint32_t>(sms) / 2;
-    const uint32_t grid = 2 * (sh.num_tiles < max_pairs ? sh.num_tiles : max_pairs);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = kSwapSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = L.pdl ? 1 : 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_swapped_kernel, tw, tt, ts, L.w_scale,
-                                       static_cast<uint16_t*>(L.y), sh);
-    note_launch();
-    return e != cudaSuccess ? e : cudaGetLastError();
-}
-
 cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream) {
     const KernelSetup& ks = setup_for_device();
     if (ks.err != cudaSuccess) return ks.err;
@@ -1334,7 +924,6 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream) {
     }
     if (L.m <= 32) return launch_decode<32, false>(L, ks.sms, stream);
     if (L.m <= kDecMaxTokens) return launch_decode<64, false>(L, ks.sms, stream);
-    if (use_swapped(L)) return launch_swapped(L, ks.sms, stream);
     CUtensorMap ta, tb, ts;
     if (!make_map_u8(&ta, L.q, L.k, L.m, BM) || !make_map_u8(&tb, L.wq, L.k, L.n, BN_CTA) ||
         !make_map_scales_box(&ts, L.s_k, L.mp, L.k / BK, BM))
