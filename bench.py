@@ -288,6 +288,60 @@ def graph_loop_ms(fn, steps: int, replays: int = 5) -> float:
     return statistics.median(times)
 
 
+E2E_DEPTH = 2  # steps in flight in the end-to-end loop (device input/output buffers per stream)
+E2E_OVERLAP = "input copy, call and result copy of consecutive steps on three streams, 2 steps in flight"
+
+
+def pipelined_e2e_ms(h2d, compute, d2h, steps: int, warmup: int) -> float:
+    """Device time per step of the end-to-end loop, as a server runs it: step
+    i's input copy (host -> device), step i-1's call and step i-2's result copy
+    (device -> host) run at once on three streams (the host link is full
+    duplex), with E2E_DEPTH device buffers per direction. Every step still
+    copies its own input in and its own result out. h2d(i, b), compute(i, b)
+    and d2h(i, b) enqueue step i's part on the current stream, using buffer b.
+    Timed with CUDA events on the calling stream, which waits for all three."""
+    import torch
+    cur = torch.cuda.current_stream()
+    s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    in_done = [torch.cuda.Event() for _ in range(E2E_DEPTH)]
+    run_done = [torch.cuda.Event() for _ in range(E2E_DEPTH)]
+    out_done = [torch.cuda.Event() for _ in range(E2E_DEPTH)]
+
+    def run(n: int, timed: bool) -> float:
+        if timed:
+            hold_stream(n)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(cur)
+        for s in (s_in, s_run, s_out):
+            s.wait_event(e0)
+        for i in range(n):
+            b = i % E2E_DEPTH
+            with torch.cuda.stream(s_in):
+                if i >= E2E_DEPTH:
+                    s_in.wait_event(run_done[b])  # the call that read input buffer b is done
+                h2d(i, b)
+                in_done[b].record(s_in)
+            with torch.cuda.stream(s_run):
+                s_run.wait_event(in_done[b])
+                if i >= E2E_DEPTH:
+                    s_run.wait_event(out_done[b])  # output buffer b has been copied out
+                compute(i, b)
+                run_done[b].record(s_run)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(run_done[b])
+                d2h(i, b)
+                out_done[b].record(s_out)
+        for s in (s_in, s_run, s_out):
+            cur.wait_stream(s)
+        e1.record(cur)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / max(1, n)
+
+    run(max(warmup, E2E_DEPTH + 1), False)
+    return run(steps, True)
+
+
 L2_BYTES = 126 * 2 ** 20
 
 
@@ -737,29 +791,22 @@ def ours_arm(args):
     clk = clocks.stop()
 
     # End to end through the public call with host buffers: pinned X in,
-    # fused linear, Y back to pinned host memory, every step.
+    # fused linear, Y back to pinned host memory, every step, with the copies
+    # of neighbouring steps overlapped (pipelined_e2e_ms).
     x_host = [torch.from_numpy(s["xb"].view(np.int16)).view(torch.bfloat16).pin_memory() for s in sets[:N_SETS]]
-    y_host = torch.empty((m, n), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty((m, k), dtype=torch.bfloat16, device=dev)
+    y_host = [torch.empty((m, n), dtype=torch.bfloat16).pin_memory() for _ in range(E2E_DEPTH)]
+    x_dev = [torch.empty((m, k), dtype=torch.bfloat16, device=dev) for _ in range(E2E_DEPTH)]
+    y_dev = [torch.empty((m, n), dtype=torch.bfloat16, device=dev) for _ in range(E2E_DEPTH)]
 
-    def e2e_step(i):
+    def e2e_compute(i, b):
         s = sets[i % n_sets]
-        x_dev.copy_(x_host[i % N_SETS], non_blocking=True)
-        linear_call(x_dev, s["wq"], s["ws"], workspace=s["work"], out=s["y"])
-        y_host.copy_(s["y"], non_blocking=True)
+        linear_call(x_dev[b], s["wq"], s["ws"], workspace=s["work"], out=y_dev[b])
 
-    for i in range(args.warmup):
-        e2e_step(i)
-    torch.cuda.synchronize()
     barrier(world)
-    hold_stream(args.steps)
-    ev0.record(stream)
-    for i in range(args.steps):
-        e2e_step(i)
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    e2e_ms = max_over_ranks(
+        pipelined_e2e_ms(lambda i, b: x_dev[b].copy_(x_host[i % N_SETS], non_blocking=True), e2e_compute,
+                         lambda i, b: y_host[b].copy_(y_dev[b], non_blocking=True), args.steps, args.warmup)
+        * args.steps, world)
 
     flops = 2.0 * m * n * k
     value = weak_scaling_value(flops, world, args.steps, ms_total) / 1e12
@@ -820,7 +867,8 @@ def ours_arm(args):
             "per_config": per_config,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": m * k * 2,
-                    "d2h_bytes_per_step": m * n * 2},
+                    "d2h_bytes_per_step": m * n * 2,
+                    "overlap": E2E_OVERLAP},
             "gpu_launches": int(sum_over_ranks(launches, world)),
             "clocks": clk,
         }
@@ -961,16 +1009,19 @@ def ffn_arm(args):
     clk = clocks.stop()
 
     x_host = [torch.from_numpy(s["xb"].view(np.int16)).view(torch.bfloat16).pin_memory() for s in sets]
-    y_host = torch.empty((m, d), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty((m, d), dtype=torch.bfloat16, device=dev)
+    y_host = [torch.empty((m, d), dtype=torch.bfloat16).pin_memory() for _ in range(E2E_DEPTH)]
+    x_dev = [torch.empty((m, d), dtype=torch.bfloat16, device=dev) for _ in range(E2E_DEPTH)]
+    y_dev = [torch.empty((m, d), dtype=torch.bfloat16, device=dev) for _ in range(E2E_DEPTH)]
 
-    def e2e(j):
+    def e2e(j, b):
         s = sets[j % N_SETS]
-        x_dev.copy_(x_host[j % N_SETS], non_blocking=True)
-        api.ffn(x_dev, *s["w"], workspace=s["work"], out=s["y"])
-        y_host.copy_(s["y"], non_blocking=True)
+        api.ffn(x_dev[b], *s["w"], workspace=s["work"], out=y_dev[b])
 
-    e2e_ms = timed(e2e, args.steps)
+    barrier(world)
+    e2e_ms = max_over_ranks(
+        pipelined_e2e_ms(lambda j, b: x_dev[b].copy_(x_host[j % N_SETS], non_blocking=True), e2e,
+                         lambda j, b: y_host[b].copy_(y_dev[b], non_blocking=True), args.steps, args.warmup),
+        world)
 
     flops = 2.0 * m * d * 2 * i + 2.0 * m * i * d
     hbm, bf16, _, src = load_peaks()
@@ -1015,7 +1066,8 @@ def ffn_arm(args):
                                    "traffic": read_traffic("silu_mul_quant_kernel", args.workload)},
             "cpu_baseline": cpu,
             "e2e": {"value": weak_scaling_value(flops, world, 1, e2e_ms) / 1e12, "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": m * d * 2, "d2h_bytes_per_step": m * d * 2},
+                    "h2d_bytes_per_step": m * d * 2, "d2h_bytes_per_step": m * d * 2,
+                    "overlap": E2E_OVERLAP},
             "gpu_launches": int(sum_over_ranks(launches, world)),
             "clocks": clk,
         }
@@ -1129,19 +1181,19 @@ def nvfp4_arm(args):
     kt = nvfp4_timings(m, n, k, dev, hbm, bf16 * 4.0, args.steps, args.warmup)
     clk = clocks.stop()
     x_host = [torch.from_numpy(s["xb"].view(np.int16)).view(torch.bfloat16).pin_memory() for s in sets[:N_SETS]]
-    y_host = torch.empty((m, n), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty((m, k), dtype=torch.bfloat16, device=dev)
+    y_host = [torch.empty((m, n), dtype=torch.bfloat16).pin_memory() for _ in range(E2E_DEPTH)]
+    x_dev = [torch.empty((m, k), dtype=torch.bfloat16, device=dev) for _ in range(E2E_DEPTH)]
+    y_dev = [torch.empty((m, n), dtype=torch.bfloat16, device=dev) for _ in range(E2E_DEPTH)]
 
-    def e2e(j):
+    def e2e(j, b):
         s = sets[j % n_sets]
-        x_dev.copy_(x_host[j % N_SETS], non_blocking=True)
-        api.nvfp4_linear(x_dev, s["qw"], s["sfw"], s["s2w"], workspace=s["work"], out=s["y"])
-        y_host.copy_(s["y"], non_blocking=True)
+        api.nvfp4_linear(x_dev[b], s["qw"], s["sfw"], s["s2w"], workspace=s["work"], out=y_dev[b])
 
-    for j in range(args.warmup):
-        e2e(j)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(stream_loop_ms(e2e, args.steps), world)
+    barrier(world)
+    e2e_ms = max_over_ranks(
+        pipelined_e2e_ms(lambda j, b: x_dev[b].copy_(x_host[j % N_SETS], non_blocking=True), e2e,
+                         lambda j, b: y_host[b].copy_(y_dev[b], non_blocking=True), args.steps, args.warmup),
+        world)
     flops = 2.0 * m * n * k
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -1164,7 +1216,8 @@ def nvfp4_arm(args):
             "pack": kt["pack"], "linear_us": kt["linear"],
             "cpu_baseline": cpu,
             "e2e": {"value": weak_scaling_value(flops, world, 1, e2e_ms) / 1e12, "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": m * k * 2, "d2h_bytes_per_step": m * n * 2},
+                    "h2d_bytes_per_step": m * k * 2, "d2h_bytes_per_step": m * n * 2,
+                    "overlap": E2E_OVERLAP},
             "gpu_launches": int(sum_over_ranks(launches, world)),
             "clocks": clk,
         }), flush=True)
