@@ -166,8 +166,9 @@ __device__ __forceinline__ uint4 silu_mul8(const uint4 g, const uint4 u) {
     return make_uint4(h[0], h[1], h[2], h[3]);
 }
 
-// grid (ceil(G/8), m), 64 threads; octet o of CTA (bx, t) owns group
-// 8*bx + o of token t. Row t of gate starts at gate + t*ld, likewise up.
+// 1-D grid of ceil(G/8) * m CTAs of 64 threads: CTA t * ceil(G/8) + bx
+// handles token t, and its octet o owns group 8*bx + o. Row t of gate
+// starts at gate + t*ld, likewise up.
 // Waits on the grid it depends on (the gate/up projection, when launched as
 // its programmatic dependent) before loading.
 __global__ void __launch_bounds__(64) silu_mul_quant_kernel(const uint16_t* __restrict__ gate,
@@ -176,11 +177,12 @@ __global__ void __launch_bounds__(64) silu_mul_quant_kernel(const uint16_t* __re
                                                            float* __restrict__ s_k, uint32_t m, uint32_t i,
                                                            uint32_t mp) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if ((blockIdx.y * gridDim.x + blockIdx.x) + kMultiTriggerTail >= gridDim.x * gridDim.y) trigger_dependents();
+    if (blockIdx.x + kMultiTriggerTail >= gridDim.x) trigger_dependents();
     const uint32_t G = i >> 7;
+    const uint32_t gx = (G + 7) >> 3;
+    const uint32_t t = blockIdx.x / gx;
     const uint32_t lane = threadIdx.x & 7;
-    const uint32_t g = blockIdx.x * 8 + (threadIdx.x >> 3);
-    const uint32_t t = blockIdx.y;
+    const uint32_t g = (blockIdx.x - t * gx) * 8 + (threadIdx.x >> 3);
     const bool g_ok = g < G;
     uint4 a0, a1, b0, b1;
     if (g_ok) {
@@ -263,7 +265,7 @@ __global__ void __launch_bounds__(256) check_silu_mul_kernel(unsigned long long*
 cudaError_t launch_silu_mul_quant(const SiluLaunch& L, bool pdl, cudaStream_t stream) {
     const uint32_t G = L.i >> 7;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((G + 7) / 8, L.m, 1);
+    cfg.gridDim = dim3(((G + 7) / 8) * L.m, 1, 1);
     cfg.blockDim = dim3(64, 1, 1);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];

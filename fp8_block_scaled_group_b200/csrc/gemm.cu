@@ -526,8 +526,8 @@ __global__ void __launch_bounds__(FUSE ? kDecFusedThreads : kDecThreads, 2)
     constexpr uint32_t kCols = kDecBufs * NT;  // 128 or 256 TMEM columns
     const uint32_t warp = threadIdx.x >> 5;
     const uint32_t lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_ctarank();  // the cluster spans grid x: rank == K split
-    const uint32_t nb = blockIdx.y;           // weight block row
+    const uint32_t rank = cluster_ctarank();  // clusters of `split` consecutive CTAs: rank == K split
+    const uint32_t nb = blockIdx.x / sh.split;  // weight block row
     const uint32_t n0 = nb * BM;
     const uint32_t G = sh.G;
     const uint32_t kb0 = rank * G / sh.split;
@@ -894,7 +894,7 @@ cudaError_t launch_decode(const GemmLaunch& L, int sms, cudaStream_t stream) {
     const uint32_t split = decode_split(slices, sh.G, sms);
     sh.split = split;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(split, slices, 1);
+    cfg.gridDim = dim3(split * slices, 1, 1);
     cfg.blockDim = dim3(FUSE ? kDecFusedThreads : kDecThreads, 1, 1);
     cfg.dynamicSmemBytes = decode_smem_bytes<NT>();
     cfg.stream = stream;

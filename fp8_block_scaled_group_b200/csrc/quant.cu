@@ -223,13 +223,14 @@ __global__ void __launch_bounds__(kStreamThreads, kStreamCtasPerSm)
     __syncwarp();
 }
 
-// Weight blocks: grid (K/128, N/128), 256 threads. The block's 128 rows x
-// 256 bytes are 2048 16-byte chunks; thread i owns chunks i + 256 j.
+// Weight blocks: a 1-D grid of (N/128) * (K/128) CTAs of 256 threads, CTA
+// bn * (K/128) + bg quantizing block (bn, bg). The block's 128 rows x 256
+// bytes are 2048 16-byte chunks; thread i owns chunks i + 256 j.
 __global__ void __launch_bounds__(256) quant_weight_kernel(const uint16_t* __restrict__ w, uint8_t* __restrict__ wq,
                                                            float* __restrict__ w_scale, uint32_t k) {
     __shared__ float red[8];
-    const uint32_t G = gridDim.x;
-    const uint32_t bg = blockIdx.x, bn = blockIdx.y;
+    const uint32_t G = k >> 7;
+    const uint32_t bn = blockIdx.x / G, bg = blockIdx.x - bn * G;
     float f[8][8];
     float amax = 0.0f;
 #pragma unroll
@@ -406,8 +407,7 @@ cudaError_t read_clear_quant_error(uint32_t* code, cudaStream_t stream) {
 
 cudaError_t launch_quant_weight(const void* w, void* wq, float* w_scale, uint32_t n, uint32_t k,
                                 cudaStream_t stream) {
-    dim3 grid(k / 128, n / 128);
-    quant_weight_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(w), static_cast<uint8_t*>(wq),
+    quant_weight_kernel<<<(k / 128) * (n / 128), 256, 0, stream>>>(static_cast<const uint16_t*>(w), static_cast<uint8_t*>(wq),
                                                   w_scale, k);
     note_launch();
     return cudaGetLastError();
