@@ -548,8 +548,20 @@ __global__ void __launch_bounds__(FUSE ? kDecFusedThreads : kDecThreads, 2)
         sm.consumed = 0;
         fence_mbar_init();
     }
+    // The weight tiles of the first stages are requested at once, so their
+    // DRAM latency overlaps the TMEM allocation and the block barrier (and,
+    // launched as the quantizer's dependent, the quantizer itself: the weight
+    // is not written by the preceding grid, and everything before that grid
+    // had finished when it let this one launch). Each such stage's barrier
+    // is armed here with all of the stage's bytes; the token tile and its
+    // scales follow once the preceding grid has completed.
+    const uint32_t pre = sh.no_copies ? 0u : (nk < kDecStages ? nk : kDecStages);
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmW);
+        for (uint32_t it = 0; it < pre; ++it) {
+            mbar_arrive_expect_tx(&sm.full[it], FUSE ? BM * BK : BM * BK + NT * BK + NT * 4);
+            tma_load_2d(sm.w[it], &tmW, &sm.full[it], static_cast<int32_t>((kb0 + it) * BK), static_cast<int32_t>(n0));
+        }
         tma_prefetch_desc(&tmT);
         tma_prefetch_desc(&tmS);
     }
@@ -570,11 +582,19 @@ __global__ void __launch_bounds__(FUSE ? kDecFusedThreads : kDecThreads, 2)
 
     if (warp == 0) {
         if (lane == 0 && !sh.no_copies) {
+            issued = pre;  // the early weight copies are in flight
             grid_dependency_wait();
             for (uint32_t it = 0; it < nk; ++it) {
                 const uint32_t kb = kb0 + it;
                 const uint32_t s = it % kDecStages;
                 const uint32_t ph = (it / kDecStages) & 1u;
+                if (it < pre) {
+                    if (!FUSE) {
+                        tma_load_2d(sm.t[s], &tmT, &sm.full[s], static_cast<int32_t>(kb * BK), 0);
+                        tma_load_2d(sm.t_scale[s], &tmS, &sm.full[s], 0, static_cast<int32_t>(kb));
+                    }
+                    continue;
+                }
                 if (!mbar_wait(&sm.empty[s], ph ^ 1u, abort, sh.budget)) break;
                 if (FUSE) {
                     mbar_arrive_expect_tx(&sm.full[s], BM * BK);

@@ -136,26 +136,17 @@ def test_quant_act_m_zero_touches_nothing():
 
 
 def test_convert_matches_oracle_encoder_exhaustively():
-    """Every fp32 pattern in [2^-11, 448] (and its negative), plus tiny and huge values."""
-    lo = int(np.float32(2.0 ** -11).view(np.uint32))
-    hi = int(np.float32(448.0).view(np.uint32))
+    """Every fp32 bit pattern except the NaNs (both zeros, subnormals, normals,
+    +-Inf): the hardware e4m3 conversion the kernels use gives the oracle
+    encoder's code."""
     step = 1 << 25
-    for start in range(lo, hi + 1, step):
-        pats = np.arange(start, min(start + step, hi + 1), dtype=np.uint32)
-        vals = pats.view(np.float32)
-        for sign in (1.0, -1.0):
-            v = vals * np.float32(sign)
+    for lo, hi in ((0x00000000, 0x7F800000), (0x80000000, 0xFF800000)):  # +0 .. +Inf, -0 .. -Inf
+        for start in range(lo, hi + 1, step):
+            pats = np.arange(start, min(start + step, hi + 1), dtype=np.uint32)
+            v = pats.view(np.float32)
             got = api.convert_e4m3(torch.from_numpy(v).to(DEV)).cpu().numpy()
             want = oracle.e4m3_encode_array(v)
             assert np.array_equal(got, want), hex(start)
-    rng = np.random.default_rng(3)
-    extra = np.concatenate([
-        rng.uniform(0, 2.0 ** -11, 1 << 16).astype(np.float32),
-        np.array([0.0, 1e-45, 1e-40, 1.17e-38, 448.0, 448.01, 463.9, 464.0, 479.0, 480.0, 1e6, 3.4e38], np.float32),
-    ])
-    extra = np.concatenate([extra, -extra])
-    got = api.convert_e4m3(torch.from_numpy(extra).to(DEV)).cpu().numpy()
-    assert np.array_equal(got, oracle.e4m3_encode_array(extra))
 
 
 def test_division_exhaustive_against_ieee():
