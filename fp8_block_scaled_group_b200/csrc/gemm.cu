@@ -507,9 +507,13 @@ __device__ __forceinline__ void tmem_load_nt<32>(uint32_t taddr, uint32_t (&r)[3
         : "memory");
 }
 
-__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+// Four consecutive floats (16-byte aligned) from a cluster peer's shared memory.
+__device__ __forceinline__ float4 ld_shared_cluster_f32x4(uint32_t cluster_addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(cluster_addr)
+                 : "memory");
     return v;
 }
 
@@ -752,23 +756,42 @@ __global__ void __launch_bounds__(FUSE ? kDecFusedThreads : kDecThreads, 2)
         for (uint32_t i = 0; i < NT; ++i) red[i * BM + r_local] = acc[i];
     }
     cluster_sync_all();
+    // CTA `rank` owns tokens rank, rank + split, ... Thread (tq, jq) of its
+    // first four warps sums rows 4jq .. 4jq+3 of every fourth owned token:
+    // one 16-byte read per peer and token, and one 8-byte store.
     if (threadIdx.x < BM && !*abort) {
-        const uint32_t j = threadIdx.x;
+        const uint32_t jq = threadIdx.x & 31u;
+        const uint32_t tq = threadIdx.x >> 5;
+        const uint32_t j = 4u * jq;
         const uint32_t red_addr = smem_addr(red);
-        const float w_row = sh.w_per_row ? __ldg(w_s + n0 + j) : 1.0f;
-        for (uint32_t t = rank; t < sh.M; t += sh.split) {
+        const float4 w_row = sh.w_per_row ? __ldg(reinterpret_cast<const float4*>(w_s + n0 + j))
+                                          : make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+        for (uint32_t t = rank + sh.split * tq; t < sh.M; t += 4u * sh.split) {
             // Issue every peer's load before adding (independent remote
             // reads in flight together), then sum in rank order.
-            float part[kDecMaxSplit];
+            float4 part[kDecMaxSplit];
 #pragma unroll
             for (uint32_t p = 0; p < kDecMaxSplit; ++p)
-                part[p] = p < sh.split ? ld_shared_cluster_f32(mapa_shared(red_addr + (t * BM + j) * 4u, p)) : 0.0f;
-            float sum = 0.0f;
+                part[p] = p < sh.split ? ld_shared_cluster_f32x4(mapa_shared(red_addr + (t * BM + j) * 4u, p))
+                                       : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            float4 sum = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
-            for (uint32_t p = 0; p < kDecMaxSplit; ++p) sum += part[p];
-            if (sh.w_per_row) sum *= w_row;
-            __nv_bfloat16 h = __float2bfloat16_rn(sum);
-            y[static_cast<size_t>(t) * sh.N + n0 + j] = *reinterpret_cast<uint16_t*>(&h);
+            for (uint32_t p = 0; p < kDecMaxSplit; ++p) {
+                sum.x += part[p].x;
+                sum.y += part[p].y;
+                sum.z += part[p].z;
+                sum.w += part[p].w;
+            }
+            if (sh.w_per_row) {
+                sum.x *= w_row.x;
+                sum.y *= w_row.y;
+                sum.z *= w_row.z;
+                sum.w *= w_row.w;
+            }
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(sum.x, sum.y);
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(sum.z, sum.w);
+            *reinterpret_cast<uint2*>(y + static_cast<size_t>(t) * sh.N + n0 + j) =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
         }
     }
     cluster_sync_all();  // peers' partials stay in place until every CTA has read them
