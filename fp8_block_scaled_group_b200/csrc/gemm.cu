@@ -507,16 +507,6 @@ __device__ __forceinline__ void tmem_load_nt<32>(uint32_t taddr, uint32_t (&r)[3
         : "memory");
 }
 
-// Four consecutive floats (16-byte aligned) from a cluster peer's shared memory.
-__device__ __forceinline__ float4 ld_shared_cluster_f32x4(uint32_t cluster_addr) {
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(cluster_addr)
-                 : "memory");
-    return v;
-}
-
 template <uint32_t NT, bool FUSE>
 __global__ void __launch_bounds__(FUSE ? kDecFusedThreads : kDecThreads, 2)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmT,

@@ -33,7 +33,10 @@
 // The GEMM is a persistent single-CTA kernel: a CTA owns a 128 x BN output
 // tile (BN = 256, or 128 at decode widths so that more CTAs stream the
 // weight), takes K in stages of 256 elements (128 bytes a row: one
-// 128-byte swizzle atom) and issues four K = 64 MMAs per stage. Per stage
+// 128-byte swizzle atom) and issues four K = 64 MMAs per stage. When one
+// row of 128-column tiles leaves SMs idle (decode widths), K is split over
+// a cluster of up to 8 CTAs, one per SM, whose fp32 partials are summed
+// through distributed shared memory in rank order. Per stage
 // TMA brings A [128 x 128 B] and B [BN x 128 B]; two or three bulk copies
 // bring the scale atoms of the stage (2 KB per 128 rows). The MMA thread
 // copies the stage's atoms into TMEM (tcgen05.cp, 4 columns per atom, the
@@ -53,6 +56,7 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "group_quant.cuh"
@@ -224,7 +228,16 @@ struct Shape {
     uint32_t M, N, K;
     uint32_t num_m, num_tiles;
     float alpha;
+    // K split (1: persistent over tiles). With split > 1 (one 128-row tile
+    // of A, BN = 128) the grid is split x tiles CTAs in clusters of `split`:
+    // CTA `rank` of a cluster takes K stages [rank, rank + 1) * stages / split
+    // of its tile, parks its fp32 partial in shared memory, and the cluster
+    // sums the partials through distributed shared memory in rank order.
+    uint32_t split;
 };
+
+constexpr uint32_t kMaxSplit = 8;
+constexpr uint32_t kRedStride = 132;  // floats per partial row (128 + 4: 16-byte rows, staggered banks)
 
 template <uint32_t BN>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -239,6 +252,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t kt_count = sh.K / (2 * kStageKBytes);
     const size_t sf_block_bytes = static_cast<size_t>(sh.K / 64) * kSfAtomBytes;  // one 128-row block
     volatile uint32_t* abort = &sm.abort;
+    // Only the 128-column tiles split K; their A stages hold the partial.
+    static_assert(kBM * kRedStride * sizeof(float) <= sizeof(Smem<128>::a), "the partial does not fit the A stages");
+    const uint32_t split = BN == 128 ? sh.split : 1u;
+    const uint32_t rank = cluster_ctarank();  // 0 without clusters
+    const uint32_t tile0 = split > 1 ? blockIdx.x / split : blockIdx.x;
+    const uint32_t tile_step = split > 1 ? sh.num_tiles : gridDim.x;  // split: one tile per CTA
+    const uint32_t kt_begin = rank * kt_count / split;
+    const uint32_t kt_end = (rank + 1) * kt_count / split;
 
     if (threadIdx.x == 0) {
         for (uint32_t s = 0; s < C::kStages; ++s) {
@@ -273,12 +294,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             grid_dependency_wait();
             uint32_t it = 0;
             bool ok = true;
-            for (uint32_t tile = blockIdx.x; ok && tile < sh.num_tiles; tile += gridDim.x) {
+            for (uint32_t tile = tile0; ok && tile < sh.num_tiles; tile += tile_step) {
                 const uint32_t m0 = (tile % sh.num_m) * kBM;
                 const uint32_t n0 = (tile / sh.num_m) * BN;
                 const uint8_t* sfa_blk = sfa + static_cast<size_t>(m0 / 128) * sf_block_bytes;
                 const uint8_t* sfb_blk = sfb + static_cast<size_t>(n0 / 128) * sf_block_bytes;
-                for (uint32_t kt = 0; kt < kt_count; ++kt, ++it) {
+                for (uint32_t kt = kt_begin; kt < kt_end; ++kt, ++it) {
                     const uint32_t s = it % C::kStages;
                     const uint32_t ph = (it / C::kStages) & 1u;
                     if (!mbar_wait(&sm.empty[s], ph ^ 1u, abort)) {
@@ -305,13 +326,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idesc = idesc_e2m1_ue4m3(kBM, BN);
             uint32_t it = 0, local = 0;
             bool ok = true;
-            for (uint32_t tile = blockIdx.x; ok && tile < sh.num_tiles; tile += gridDim.x, ++local) {
+            for (uint32_t tile = tile0; ok && tile < sh.num_tiles; tile += tile_step, ++local) {
                 const uint32_t buf = local % C::kAccBufs;
                 const uint32_t bph = (local / C::kAccBufs) & 1u;
                 if (!mbar_wait(&sm.acc_empty[buf], bph ^ 1u, abort)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + buf * BN;
-                for (uint32_t kt = 0; kt < kt_count; ++kt, ++it) {
+                for (uint32_t kt = kt_begin; kt < kt_end; ++kt, ++it) {
                     const uint32_t s = it % C::kStages;
                     const uint32_t ph = (it / C::kStages) & 1u;
                     if (!mbar_wait(&sm.full[s], ph, abort)) {
@@ -335,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (uint32_t j = 0; j < kKSteps; ++j)
                         mma_mxf4nvf4(d, ad + 2u * j, bd + 2u * j, idesc, tmem + kSfaCol + 4u * j,
-                                     tmem + kSfbCol + 4u * C::kNBlk * j, (kt | j) != 0 ? 1u : 0u);
+                                     tmem + kSfbCol + 4u * C::kNBlk * j, (kt != kt_begin || j != 0) ? 1u : 0u);
                     mma_commit(&sm.empty[s]);
                 }
                 if (!ok) break;
@@ -350,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t quarter = warp & 3u;
         const uint32_t lane_off = (quarter * 32u) << 16;
         uint32_t local = 0;
-        for (uint32_t tile = blockIdx.x; tile < sh.num_tiles; tile += gridDim.x, ++local) {
+        for (uint32_t tile = tile0; tile < sh.num_tiles; tile += tile_step, ++local) {
             const uint32_t m0 = (tile % sh.num_m) * kBM;
             const uint32_t n0 = (tile / sh.num_m) * BN;
             const uint32_t buf = local % C::kAccBufs;
@@ -359,6 +380,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!__all_sync(0xFFFFFFFFu, got)) break;
             tc_fence_after();
             const uint32_t row = m0 + quarter * 32u + lane;
+            if (split > 1) {
+                // The partial, fp32, into the idle A stages (every MMA of
+                // this CTA has completed): red[row][column].
+                float* red = reinterpret_cast<float*>(&sm.a[0][0]);
+#pragma unroll 1
+                for (uint32_t c = 0; c < BN / 64; ++c) {
+                    uint32_t v[64];
+                    tmem_load64(tmem + lane_off + buf * BN + c * 64u, v);
+                    if (row < sh.M) {
+                        float4* dst = reinterpret_cast<float4*>(red + row * kRedStride + c * 64u);
+#pragma unroll
+                        for (uint32_t j = 0; j < 16; ++j)
+                            dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+                    }
+                }
+                continue;
+            }
 #pragma unroll 1
             for (uint32_t c = 0; c < BN / 64; ++c) {
                 uint32_t v[64];
@@ -400,6 +439,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
+    }
+
+    if (split > 1) {
+        // CTA `rank` owns tokens rank, rank + split, ...; thread (tq, jq) of
+        // its first four warps sums columns 4jq .. 4jq+3 of every fourth
+        // owned token over the cluster in rank order, one 16-byte read per
+        // peer, scales by alpha and stores four bf16 outputs.
+        cluster_sync_all();
+        if (threadIdx.x < 128 && !*abort) {
+            const uint32_t jq = threadIdx.x & 31u;
+            const uint32_t tq = threadIdx.x >> 5;
+            const uint32_t j = 4u * jq;
+            const uint32_t n0 = tile0 * BN;
+            const uint32_t red_addr = smem_addr(&sm.a[0][0]);
+            for (uint32_t t = rank + split * tq; t < sh.M; t += 4u * split) {
+                float4 part[kMaxSplit];
+#pragma unroll
+                for (uint32_t p = 0; p < kMaxSplit; ++p)
+                    part[p] = p < split ? ld_shared_cluster_f32x4(mapa_shared(red_addr + (t * kRedStride + j) * 4u, p))
+                                        : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                float4 sum = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+                for (uint32_t p = 0; p < kMaxSplit; ++p) {
+                    sum.x += part[p].x;
+                    sum.y += part[p].y;
+                    sum.z += part[p].z;
+                    sum.w += part[p].w;
+                }
+                const __nv_bfloat162 lo = __floats2bfloat162_rn(sh.alpha * sum.x, sh.alpha * sum.y);
+                const __nv_bfloat162 hi = __floats2bfloat162_rn(sh.alpha * sum.z, sh.alpha * sum.w);
+                *reinterpret_cast<uint2*>(y + static_cast<size_t>(t) * sh.N + n0 + j) =
+                    make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+            }
+        }
+        cluster_sync_all();  // peers' partials stay in place until every CTA has read them
     }
 }
 
@@ -459,6 +533,36 @@ const Setup& setup_for_device() {
     return s;
 }
 
+// Clusters of `split` 128-column-tile CTAs that fit the GPU at once, per
+// device and split (cached).
+int fitting_clusters(uint32_t split) {
+    static std::mutex mu;
+    static int table[64][kMaxSplit + 1] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    int& n = table[dev][split];
+    if (n == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(split * 64, 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem_bytes<128>();
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = split;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, nvfp4_gemm_kernel<128>, &cfg) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = -1;  // unknown: do not split
+        }
+    }
+    return n;
+}
+
 unsigned grid_for(uint64_t items, int sms) {
     uint64_t blocks = (items + 255) / 256;
     const uint64_t cap = static_cast<uint64_t>(sms > 0 ? sms : 148) * 16u;
@@ -478,17 +582,57 @@ cudaError_t launch_gemm_bn(const Nvfp4GemmLaunch& L, int sms, cudaStream_t strea
     sh.num_m = (L.m + kBM - 1) / kBM;
     sh.num_tiles = sh.num_m * (L.n / BN);
     sh.alpha = L.alpha;
-    const uint32_t grid = sh.num_tiles < static_cast<uint32_t>(sms) ? sh.num_tiles : static_cast<uint32_t>(sms);
+    // One row of 128-column tiles with fewer tiles than SMs (decode
+    // widths): split K so that more SMs stream the weight (one CTA per SM,
+    // at most kMaxSplit per cluster, at least one K stage each), taking the
+    // largest split whose clusters all fit the GPU at once.
+    const uint32_t kt_count = L.k / (2 * kStageKBytes);
+    uint32_t split = 1;
+    if (BN == 128 && sh.num_m == 1) {
+        uint32_t s = static_cast<uint32_t>(sms) / sh.num_tiles;
+        if (s > kMaxSplit) s = kMaxSplit;
+        if (s > kt_count) s = kt_count;
+        for (; s > 1; --s) {
+            const int fit = fitting_clusters(s);
+            if (fit > 0 && static_cast<uint32_t>(fit) >= sh.num_tiles) break;
+        }
+        split = s < 1 ? 1 : s;
+        // FP8Q_NVFP4_SPLIT=<n> overrides the choice (sweeps).
+        static const int forced = [] {
+            const char* e = std::getenv("FP8Q_NVFP4_SPLIT");
+            return e ? std::atoi(e) : 0;
+        }();
+        if (forced > 0) {
+            split = static_cast<uint32_t>(forced);
+            if (split > kMaxSplit) split = kMaxSplit;
+            if (split > kt_count) split = kt_count;
+        }
+    }
+    sh.split = split;
+    const uint32_t grid = split > 1 ? split * sh.num_tiles
+                                    : (sh.num_tiles < static_cast<uint32_t>(sms) ? sh.num_tiles
+                                                                                 : static_cast<uint32_t>(sms));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem_bytes<BN>();
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    uint32_t na = 0;
+    if (split > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = split;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (L.pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = L.pdl ? 1 : 0;
+    cfg.numAttrs = na;
     cudaError_t e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<BN>, ta, tb, static_cast<const uint8_t*>(L.sfa),
                                        static_cast<const uint8_t*>(L.sfw), static_cast<uint16_t*>(L.y), sh);
     note_launch();

@@ -344,6 +344,16 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
                  : "memory");
 }
 
+// Four consecutive floats (16-byte aligned) from a cluster peer's shared memory.
+__device__ __forceinline__ float4 ld_shared_cluster_f32x4(uint32_t cluster_addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(cluster_addr)
+                 : "memory");
+    return v;
+}
+
 // Full barrier across the cluster (all threads of every CTA).
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");

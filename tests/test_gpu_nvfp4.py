@@ -120,7 +120,10 @@ def gemm_case(m, n, k, seed, rows=None):
 
 
 @pytest.mark.parametrize("m,n,k", [(1, 128, 256), (17, 256, 512), (128, 384, 256), (129, 512, 1024),
-                                   (300, 768, 2048), (256, 256, 5120)])
+                                   (300, 768, 2048), (256, 256, 5120),
+                                   # one row of 128-column tiles: K split over clusters of 5, 8 and 8
+                                   # CTAs, with K stages that do not divide evenly
+                                   (64, 1024, 1280), (33, 2048, 3584), (128, 768, 5120)])
 def test_nvfp4_gemm_full(m, n, k):
     bad, worst = gemm_case(m, n, k, seed=m + n + k)
     assert bad == 0, f"{bad} elements out of tolerance (worst {worst:.3f})"
