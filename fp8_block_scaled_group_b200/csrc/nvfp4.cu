@@ -47,9 +47,11 @@
 //   warp 1     TMEM allocation; MMA issuer (one thread)
 //   warps 2-5  epilogue: warp w reads TMEM lanes 32*(w%4)..+31 (tile rows),
 //              scales by alpha, rounds to bf16 and stores its rows
-// TMEM: accumulator buffers at columns 0..255 (one of 256 columns for
-// BN = 256, two of 128 for BN = 128), A scales at 256..271 (4 columns per
-// K = 64 step), B scales from 272 (4 columns per 128 rows per step).
+// TMEM: accumulator buffers from column 0 (one of 256 columns for
+// BN = 256, two of 128 for BN = 128, one of 128 for decode widths' 32-row A
+// stages), then the A scales (4 columns per K = 64 step) and the B scales
+// (4 columns per 128 rows per step); 512 columns allocated, or 256 at
+// decode widths so that two CTAs share an SM.
 // Every mbarrier wait is bounded; a CTA that gives up sets bit 1 of this
 // file's error word and winds down.
 #include <cuda.h>
@@ -188,29 +190,36 @@ constexpr uint32_t kKSteps = 4;                              // K = 64 MMAs per 
 constexpr uint32_t kSfStageBytes = kKSteps * kSfAtomBytes;   // one 128-row block's scales per stage
 constexpr uint32_t kThreads = 192;
 constexpr uint32_t kEpiWarps = 4;
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSfaCol = 256;
-constexpr uint32_t kSfbCol = kSfaCol + 4 * kKSteps;
 
-template <uint32_t BN>
+// AR: rows of A each stage holds. 128 in general; 32 when all of M fits in
+// 32 rows (decode widths), so that a stage takes 24 KB and two CTAs fit an
+// SM. The MMA still reads 128 rows of A: rows 32..127 come from whatever
+// the shared memory after the stage holds, finite E2M1 codes whose scale
+// factors are the zero pad rows of the A scales, and they only feed output
+// rows that are never stored.
+template <uint32_t BN, uint32_t AR>
 struct Cfg {
-    static constexpr uint32_t kStages = BN == 256 ? 4 : 6;
-    static constexpr uint32_t kAccBufs = BN == 256 ? 1 : 2;
+    static constexpr uint32_t kStages = BN == 256 ? 4 : (AR == 32 ? 4 : 6);
+    // One accumulator buffer at AR = 32, so that the allocation (256
+    // columns) lets two CTAs share an SM's tensor memory.
+    static constexpr uint32_t kAccBufs = BN == 256 || AR == 32 ? 1 : 2;
     static constexpr uint32_t kNBlk = BN / 128;  // 128-row scale blocks of B per tile
     static constexpr uint32_t kSfbBytes = kNBlk * kSfStageBytes;
-    static constexpr uint32_t kStageTx = kBM * kStageKBytes + BN * kStageKBytes + kSfStageBytes + kSfbBytes;
-    static_assert(kAccBufs * BN <= kSfaCol, "accumulators overlap the scale columns");
+    static constexpr uint32_t kStageTx = AR * kStageKBytes + BN * kStageKBytes + kSfStageBytes + kSfbBytes;
+    static constexpr uint32_t kSfaCol = kAccBufs * BN;  // A scales: 4 columns per K = 64 step
+    static constexpr uint32_t kSfbCol = kSfaCol + 4 * kKSteps;
+    static constexpr uint32_t kTmemCols = kSfbCol + 4 * kNBlk * kKSteps <= 256 ? 256 : 512;
     static_assert(kSfbCol + 4 * kNBlk * kKSteps <= kTmemCols, "scale columns exceed the allocation");
 };
 
-template <uint32_t BN>
+template <uint32_t BN, uint32_t AR>
 struct __align__(1024) Smem {
-    uint8_t a[Cfg<BN>::kStages][kBM * kStageKBytes];
-    uint8_t b[Cfg<BN>::kStages][BN * kStageKBytes];
-    uint8_t sfa[Cfg<BN>::kStages][kSfStageBytes];
-    uint8_t sfb[Cfg<BN>::kStages][Cfg<BN>::kSfbBytes];
-    uint64_t full[Cfg<BN>::kStages];
-    uint64_t empty[Cfg<BN>::kStages];
+    uint8_t a[Cfg<BN, AR>::kStages][AR * kStageKBytes];
+    uint8_t b[Cfg<BN, AR>::kStages][BN * kStageKBytes];
+    uint8_t sfa[Cfg<BN, AR>::kStages][kSfStageBytes];
+    uint8_t sfb[Cfg<BN, AR>::kStages][Cfg<BN, AR>::kSfbBytes];
+    uint64_t full[Cfg<BN, AR>::kStages];
+    uint64_t empty[Cfg<BN, AR>::kStages];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t mma_done;
@@ -219,9 +228,9 @@ struct __align__(1024) Smem {
     uint32_t consumed;
 };
 
-template <uint32_t BN>
+template <uint32_t BN, uint32_t AR>
 constexpr size_t smem_bytes() {
-    return sizeof(Smem<BN>) + 1024;  // + alignment slack
+    return sizeof(Smem<BN, AR>) + 1024;  // + alignment slack
 }
 
 struct Shape {
@@ -239,21 +248,23 @@ struct Shape {
 constexpr uint32_t kMaxSplit = 8;
 constexpr uint32_t kRedStride = 132;  // floats per partial row (128 + 4: 16-byte rows, staggered banks)
 
-template <uint32_t BN>
+template <uint32_t BN, uint32_t AR>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb, uint16_t* __restrict__ y,
                       const Shape sh) {
-    using C = Cfg<BN>;
+    using C = Cfg<BN, AR>;
     extern __shared__ uint8_t smem_raw[];
-    Smem<BN>& sm = *reinterpret_cast<Smem<BN>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Smem<BN, AR>& sm =
+        *reinterpret_cast<Smem<BN, AR>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t warp = threadIdx.x >> 5;
     const uint32_t lane = threadIdx.x & 31;
     const uint32_t kt_count = sh.K / (2 * kStageKBytes);
     const size_t sf_block_bytes = static_cast<size_t>(sh.K / 64) * kSfAtomBytes;  // one 128-row block
     volatile uint32_t* abort = &sm.abort;
-    // Only the 128-column tiles split K; their A stages hold the partial.
-    static_assert(kBM * kRedStride * sizeof(float) <= sizeof(Smem<128>::a), "the partial does not fit the A stages");
+    // Only the 128-column tiles split K; their B stages hold the partial
+    // (at most AR rows).
+    static_assert(BN != 128 || AR * kRedStride * sizeof(float) <= sizeof(sm.b), "the partial does not fit the B stages");
     const uint32_t split = BN == 128 ? sh.split : 1u;
     const uint32_t rank = cluster_ctarank();  // 0 without clusters
     const uint32_t tile0 = split > 1 ? blockIdx.x / split : blockIdx.x;
@@ -280,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmB);
     }
     if (warp == 1) {
-        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_alloc(&sm.tmem_base, C::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -345,18 +356,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t sfb_s = smem_addr(sm.sfb[s]);
 #pragma unroll
                     for (uint32_t j = 0; j < kKSteps; ++j) {
-                        tmem_copy_sf_atom(tmem + kSfaCol + 4u * j, smem_desc_sf_atom(sfa_s + j * kSfAtomBytes));
+                        tmem_copy_sf_atom(tmem + C::kSfaCol + 4u * j, smem_desc_sf_atom(sfa_s + j * kSfAtomBytes));
 #pragma unroll
                         for (uint32_t nb = 0; nb < C::kNBlk; ++nb)
-                            tmem_copy_sf_atom(tmem + kSfbCol + 4u * (j * C::kNBlk + nb),
+                            tmem_copy_sf_atom(tmem + C::kSfbCol + 4u * (j * C::kNBlk + nb),
                                               smem_desc_sf_atom(sfb_s + nb * kSfStageBytes + j * kSfAtomBytes));
                     }
                     const uint64_t ad = smem_desc_k_sw128(smem_addr(sm.a[s]));
                     const uint64_t bd = smem_desc_k_sw128(smem_addr(sm.b[s]));
 #pragma unroll
                     for (uint32_t j = 0; j < kKSteps; ++j)
-                        mma_mxf4nvf4(d, ad + 2u * j, bd + 2u * j, idesc, tmem + kSfaCol + 4u * j,
-                                     tmem + kSfbCol + 4u * C::kNBlk * j, (kt != kt_begin || j != 0) ? 1u : 0u);
+                        mma_mxf4nvf4(d, ad + 2u * j, bd + 2u * j, idesc, tmem + C::kSfaCol + 4u * j,
+                                     tmem + C::kSfbCol + 4u * C::kNBlk * j, (kt != kt_begin || j != 0) ? 1u : 0u);
                     mma_commit(&sm.empty[s]);
                 }
                 if (!ok) break;
@@ -381,9 +392,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const uint32_t row = m0 + quarter * 32u + lane;
             if (split > 1) {
-                // The partial, fp32, into the idle A stages (every MMA of
+                // The partial, fp32, into the idle B stages (every MMA of
                 // this CTA has completed): red[row][column].
-                float* red = reinterpret_cast<float*>(&sm.a[0][0]);
+                float* red = reinterpret_cast<float*>(&sm.b[0][0]);
 #pragma unroll 1
                 for (uint32_t c = 0; c < BN / 64; ++c) {
                     uint32_t v[64];
@@ -438,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, C::kTmemCols);
     }
 
     if (split > 1) {
@@ -452,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t tq = threadIdx.x >> 5;
             const uint32_t j = 4u * jq;
             const uint32_t n0 = tile0 * BN;
-            const uint32_t red_addr = smem_addr(&sm.a[0][0]);
+            const uint32_t red_addr = smem_addr(&sm.b[0][0]);
             for (uint32_t t = rank + split * tq; t < sh.M; t += 4u * split) {
                 float4 part[kMaxSplit];
 #pragma unroll
@@ -523,44 +534,17 @@ const Setup& setup_for_device() {
     Setup& s = table[dev];
     if (!done[dev]) {
         done[dev] = true;
-        s.err = cudaFuncSetAttribute(nvfp4_gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(smem_bytes<256>()));
+        s.err = cudaFuncSetAttribute(nvfp4_gemm_kernel<256, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem_bytes<256, 128>()));
         if (s.err == cudaSuccess)
-            s.err = cudaFuncSetAttribute(nvfp4_gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem_bytes<128>()));
+            s.err = cudaFuncSetAttribute(nvfp4_gemm_kernel<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem_bytes<128, 128>()));
+        if (s.err == cudaSuccess)
+            s.err = cudaFuncSetAttribute(nvfp4_gemm_kernel<128, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem_bytes<128, 32>()));
         if (s.err == cudaSuccess) s.err = cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev);
     }
     return s;
-}
-
-// Clusters of `split` 128-column-tile CTAs that fit the GPU at once, per
-// device and split (cached).
-int fitting_clusters(uint32_t split) {
-    static std::mutex mu;
-    static int table[64][kMaxSplit + 1] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) dev = 0;
-    std::lock_guard<std::mutex> lock(mu);
-    int& n = table[dev][split];
-    if (n == 0) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(split * 64, 1, 1);
-        cfg.blockDim = dim3(kThreads, 1, 1);
-        cfg.dynamicSmemBytes = smem_bytes<128>();
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = split;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if (cudaOccupancyMaxActiveClusters(&n, nvfp4_gemm_kernel<128>, &cfg) != cudaSuccess || n < 1) {
-            cudaGetLastError();
-            n = -1;  // unknown: do not split
-        }
-    }
-    return n;
 }
 
 unsigned grid_for(uint64_t items, int sms) {
@@ -570,10 +554,10 @@ unsigned grid_for(uint64_t items, int sms) {
     return static_cast<unsigned>(blocks ? blocks : 1);
 }
 
-template <uint32_t BN>
+template <uint32_t BN, uint32_t AR>
 cudaError_t launch_gemm_bn(const Nvfp4GemmLaunch& L, int sms, cudaStream_t stream) {
     CUtensorMap ta, tb;
-    if (!make_map_packed(&ta, L.qa, L.k / 2, L.m, kBM) || !make_map_packed(&tb, L.qw, L.k / 2, L.n, BN))
+    if (!make_map_packed(&ta, L.qa, L.k / 2, L.m, AR) || !make_map_packed(&tb, L.qw, L.k / 2, L.n, BN))
         return cudaErrorInvalidValue;
     Shape sh;
     sh.M = L.m;
@@ -583,19 +567,20 @@ cudaError_t launch_gemm_bn(const Nvfp4GemmLaunch& L, int sms, cudaStream_t strea
     sh.num_tiles = sh.num_m * (L.n / BN);
     sh.alpha = L.alpha;
     // One row of 128-column tiles with fewer tiles than SMs (decode
-    // widths): split K so that more SMs stream the weight (one CTA per SM,
-    // at most kMaxSplit per cluster, at least one K stage each), taking the
-    // largest split whose clusters all fit the GPU at once.
+    // widths): split K so that more SMs stream the weight, aiming at 0.8
+    // CTA per SM-slot in total (1.6 per SM with 32-row A stages, which fit
+    // two to an SM; 0.8 otherwise), at most kMaxSplit per cluster and at
+    // least one K stage each. Measured on B200 at M=25, N=6144, K=5120
+    // (48 tiles): 32-row stages ran 11.4 / 10.3 / 9.9 / 9.6 / 14.3 us at
+    // splits 2 / 3 / 4 / 5 / 6 (5 chosen); 128-row stages 15.5 / 11.7 /
+    // 17.5 us at 1 / 2 / 3 (2 chosen). Larger splits no longer fit at once.
     const uint32_t kt_count = L.k / (2 * kStageKBytes);
     uint32_t split = 1;
     if (BN == 128 && sh.num_m == 1) {
-        uint32_t s = static_cast<uint32_t>(sms) / sh.num_tiles;
+        const float target = (AR == 32 ? 1.6f : 0.8f) * static_cast<float>(sms);
+        uint32_t s = static_cast<uint32_t>(target / static_cast<float>(sh.num_tiles) + 0.5f);
         if (s > kMaxSplit) s = kMaxSplit;
         if (s > kt_count) s = kt_count;
-        for (; s > 1; --s) {
-            const int fit = fitting_clusters(s);
-            if (fit > 0 && static_cast<uint32_t>(fit) >= sh.num_tiles) break;
-        }
         split = s < 1 ? 1 : s;
         // FP8Q_NVFP4_SPLIT=<n> overrides the choice (sweeps).
         static const int forced = [] {
@@ -609,13 +594,12 @@ cudaError_t launch_gemm_bn(const Nvfp4GemmLaunch& L, int sms, cudaStream_t strea
         }
     }
     sh.split = split;
-    const uint32_t grid = split > 1 ? split * sh.num_tiles
-                                    : (sh.num_tiles < static_cast<uint32_t>(sms) ? sh.num_tiles
-                                                                                 : static_cast<uint32_t>(sms));
+    const uint32_t slots = (AR == 32 ? 2u : 1u) * static_cast<uint32_t>(sms);  // CTAs resident at once
+    const uint32_t grid = split > 1 ? split * sh.num_tiles : (sh.num_tiles < slots ? sh.num_tiles : slots);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem_bytes<BN>();
+    cfg.dynamicSmemBytes = smem_bytes<BN, AR>();
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     uint32_t na = 0;
@@ -633,7 +617,7 @@ cudaError_t launch_gemm_bn(const Nvfp4GemmLaunch& L, int sms, cudaStream_t strea
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<BN>, ta, tb, static_cast<const uint8_t*>(L.sfa),
+    cudaError_t e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<BN, AR>, ta, tb, static_cast<const uint8_t*>(L.sfa),
                                        static_cast<const uint8_t*>(L.sfw), static_cast<uint16_t*>(L.y), sh);
     note_launch();
     return e != cudaSuccess ? e : cudaGetLastError();
@@ -668,8 +652,10 @@ cudaError_t launch_nvfp4_gemm(const Nvfp4GemmLaunch& L, cudaStream_t stream) {
     if (s.err != cudaSuccess) return s.err;
     // One 128-row tile of A (decode widths): 128-column tiles, so that twice
     // as many CTAs stream the weight. Otherwise 256 columns where N allows.
-    if (L.m <= kBM || L.n % 256u != 0) return launch_gemm_bn<128>(L, s.sms, stream);
-    return launch_gemm_bn<256>(L, s.sms, stream);
+    // Decode widths (M <= 32): 32-row A stages, two CTAs per SM.
+    if (L.m <= 32) return launch_gemm_bn<128, 32>(L, s.sms, stream);
+    if (L.m <= kBM || L.n % 256u != 0) return launch_gemm_bn<128, 128>(L, s.sms, stream);
+    return launch_gemm_bn<256, 128>(L, s.sms, stream);
 }
 
 cudaError_t launch_convert_e2m1(const float* in, uint8_t* out, size_t n, cudaStream_t stream) {

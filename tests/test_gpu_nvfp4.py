@@ -123,7 +123,9 @@ def gemm_case(m, n, k, seed, rows=None):
                                    (300, 768, 2048), (256, 256, 5120),
                                    # one row of 128-column tiles: K split over clusters of 5, 8 and 8
                                    # CTAs, with K stages that do not divide evenly
-                                   (64, 1024, 1280), (33, 2048, 3584), (128, 768, 5120)])
+                                   (64, 1024, 1280), (33, 2048, 3584), (128, 768, 5120),
+                                   # M <= 32: 32-row A stages, split (2) and persistent (400 tiles)
+                                   (32, 1024, 1280), (8, 51200, 256)])
 def test_nvfp4_gemm_full(m, n, k):
     bad, worst = gemm_case(m, n, k, seed=m + n + k)
     assert bad == 0, f"{bad} elements out of tolerance (worst {worst:.3f})"
