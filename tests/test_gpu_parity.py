@@ -199,7 +199,9 @@ def gemm_case(m, n, k, seed, p=0.01, sigma=20.0, rows=None, threads=8):
 
 
 @pytest.mark.parametrize("m,n,k", [(1, 128, 128), (16, 512, 512), (17, 128, 640), (100, 256, 256),
-                                   (128, 384, 384), (129, 128, 1024), (200, 640, 896), (256, 256, 2048)])
+                                   (128, 384, 384), (129, 128, 1024), (200, 640, 896), (256, 256, 2048),
+                                   # 64-token decode tiles, and the first width on the pair kernel
+                                   (33, 256, 512), (48, 1024, 3072), (64, 384, 1152), (65, 256, 256)])
 def test_gemm_edges_full(m, n, k):
     bad, worst, _, _ = gemm_case(m, n, k, seed=m + n + k)
     assert bad == 0, f"{bad} elements out of tolerance (worst {worst:.3f})"
