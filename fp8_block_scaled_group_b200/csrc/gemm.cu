@@ -77,9 +77,15 @@ constexpr uint32_t kRegsLow = 40;
 constexpr uint32_t kRegsHigh = 232;
 constexpr uint32_t kLaunchRegsNeeded = (128 * kRegsLow + 256 * kRegsHigh) / kThreads;
 
+// Output staging: per promotion warp, one 32-row x 32-column bf16 block
+// (64-byte rows, 64-byte swizzle) that a TMA store writes to y.
+constexpr uint32_t kOutCols = 32;
+constexpr uint32_t kOutStageBytes = 32 * kOutCols * 2;
+
 struct __align__(1024) GemmSmem {
     uint8_t a[kStages][kTileBytesA];
     uint8_t b[kStages][kTileBytesB];
+    uint8_t out[kEpiWarps][kOutStageBytes];
     float a_scale[kScaleStages][BM];
     uint64_t full[kStages];
     uint64_t empty[kStages];
@@ -134,8 +140,8 @@ constexpr uint32_t kDirectScalesMaxG = 64;
 template <bool kDirect>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_blockscaled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                            const __grid_constant__ CUtensorMap tmS, const float* __restrict__ s_k,
-                            const float* __restrict__ w_s, uint16_t* __restrict__ y, const Shape sh) {
+                            const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmY,
+                            const float* __restrict__ s_k, const float* __restrict__ w_s, const Shape sh) {
     extern __shared__ uint8_t smem_raw[];
     GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t warp = threadIdx.x >> 5;
@@ -168,6 +174,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
         if (!kDirect) tma_prefetch_desc(&tmS);
+        tma_prefetch_desc(&tmY);
     }
     if (warp == 1) {
         tmem_alloc_pair(&sm.tmem_base, kTmemCols);
@@ -350,7 +357,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     if constexpr (!kDirect) mbar_arrive(&sm.sempty[ss]);
                 }
             }
-            if (ok && row_ok && col_ok) {
+            // Warps whose 32 rows all lie past M have nothing to store.
+            if (ok && col_ok && m0 + rank * BM + quad * 32u < sh.M) {
                 if (per_row) {
                     const float4* wv = reinterpret_cast<const float4*>(w_s + col0);
 #pragma unroll
@@ -360,19 +368,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         acc[2 * j + 1] = __fmul2_rn(acc[2 * j + 1], make_float2(v.z, v.w));
                     }
                 }
-                uint4* dst = reinterpret_cast<uint4*>(y + static_cast<size_t>(row) * sh.N + col0);
+                // The warp's 32 rows x 128 columns leave as four 32 x 32
+                // bf16 blocks: each lane packs its row of a block into the
+                // warp's staging buffer (16-byte chunk j of row r at chunk
+                // j ^ ((r >> 1) & 3), the 64-byte swizzle of the output map),
+                // and lane 0 stores the block with TMA, asynchronously, so the
+                // warps go on to the next tile's promotion. Rows past M are
+                // clipped by the map.
+                uint8_t* stg = sm.out[warp - 4u];
+                const int32_t y_row = static_cast<int32_t>(m0 + rank * BM + quad * 32u);
 #pragma unroll
-                for (uint32_t j = 0; j < 16; ++j) {
-                    uint32_t p[4];
+                for (uint32_t c = 0; c < 128u / kOutCols; ++c) {
+                    if (lane == 0) bulk_store_wait_read();  // the block before has left the buffer
+                    __syncwarp();
 #pragma unroll
-                    for (uint32_t e = 0; e < 4; ++e) {
-                        __nv_bfloat162 h = __floats2bfloat162_rn(acc[4 * j + e].x, acc[4 * j + e].y);
-                        p[e] = *reinterpret_cast<uint32_t*>(&h);
+                    for (uint32_t j = 0; j < 4; ++j) {
+                        uint32_t p[4];
+#pragma unroll
+                        for (uint32_t e = 0; e < 4; ++e) {
+                            const float2 v = acc[16 * c + 4 * j + e];
+                            __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+                            p[e] = *reinterpret_cast<uint32_t*>(&h);
+                        }
+                        *reinterpret_cast<uint4*>(stg + lane * 64u + ((j ^ ((lane >> 1) & 3u)) << 4)) =
+                            make_uint4(p[0], p[1], p[2], p[3]);
                     }
-                    dst[j] = make_uint4(p[0], p[1], p[2], p[3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) tma_store_2d(&tmY, stg, static_cast<int32_t>(col0 + c * kOutCols), y_row);
                 }
             }
         }
+        // Every output block of this warp is in global memory before the CTA
+        // (and its staging buffer) goes away.
+        if (lane == 0) bulk_store_wait_all();
+        __syncwarp();
     }
 
     // Teardown. On the normal path every TMA load was consumed and every MMA
@@ -817,6 +847,21 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t ro
     return r == CUDA_SUCCESS;
 }
 
+// The bf16 output y [rows, cols] written in [32 x 32] blocks with the
+// 64-byte swizzle (the GEMM epilogue's staging layout).
+bool make_map_out_bf16(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {kOutCols, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // The K-major activation scales [G, Mp] fp32 read as [1 x box] row slices
 // (box tokens of one K group); tokens past Mp read as zero.
 bool make_map_scales_box(CUtensorMap* map, const float* base, uint64_t mp, uint64_t g, uint32_t box_tokens) {
@@ -957,9 +1002,9 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream) {
     }
     if (L.m <= 32) return launch_decode<32, false>(L, ks.sms, stream);
     if (L.m <= kDecMaxTokens) return launch_decode<64, false>(L, ks.sms, stream);
-    CUtensorMap ta, tb, ts;
+    CUtensorMap ta, tb, ts, ty;
     if (!make_map_u8(&ta, L.q, L.k, L.m, BM) || !make_map_u8(&tb, L.wq, L.k, L.n, BN_CTA) ||
-        !make_map_scales_box(&ts, L.s_k, L.mp, L.k / BK, BM))
+        !make_map_scales_box(&ts, L.s_k, L.mp, L.k / BK, BM) || !make_map_out_bf16(&ty, L.y, L.n, L.m))
         return cudaErrorInvalidValue;
     Shape sh;
     sh.M = L.m;
@@ -984,10 +1029,8 @@ cudaError_t launch_gemm(const GemmLaunch& L, cudaStream_t stream) {
     cfg.attrs = attr;
     cfg.numAttrs = L.pdl ? 1 : 0;
     const bool direct = sh.G <= kDirectScalesMaxG;
-    cudaError_t e = direct ? cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<true>, ta, tb, ts, L.s_k, L.w_scale,
-                                                static_cast<uint16_t*>(L.y), sh)
-                           : cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<false>, ta, tb, ts, L.s_k, L.w_scale,
-                                                static_cast<uint16_t*>(L.y), sh);
+    cudaError_t e = direct ? cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<true>, ta, tb, ts, ty, L.s_k, L.w_scale, sh)
+                           : cudaLaunchKernelEx(&cfg, gemm_blockscaled_kernel<false>, ta, tb, ts, ty, L.s_k, L.w_scale, sh);
     note_launch();
     return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -127,6 +127,17 @@ __device__ __forceinline__ void bulk_store(void* dst, const void* smem_src, uint
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
+// 2-D tiled store shared -> global through a tensor map (box from the map,
+// elements outside the tensor not written), tracked in this thread's bulk
+// async-group. x is the innermost coordinate; neither may be negative.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_addr(smem_src)), "r"(x), "r"(y)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
 // Wait until this thread's bulk stores have finished reading shared memory.
 __device__ __forceinline__ void bulk_store_wait_read() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
