@@ -100,12 +100,22 @@ KERNEL_SOURCES = {
 FP8_NOMINAL_TFLOPS = 4500.0
 
 
+def strip_comments(src: str) -> str:
+    """C/C++ source without its comments and with whitespace runs collapsed,
+    so that editing a comment does not change a kernel's digest."""
+    import re
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
 def kernel_digest(kernel: str) -> str:
+    """Digest of the code (comments stripped) of a kernel's source files."""
     import hashlib
     h = hashlib.sha256()
     for name in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(ROOT, "fp8_block_scaled_group_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "fp8_block_scaled_group_b200", "csrc", name), encoding="utf-8") as f:
+            h.update(strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

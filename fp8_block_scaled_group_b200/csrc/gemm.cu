@@ -31,10 +31,12 @@
 //   warp 3      idle after set-up
 //   warps 4-11  promotion + epilogue. Warp w reads TMEM lanes 32*(w%4)..+31
 //               of its own CTA (its tile rows) and column half (w-4)/4 (128
-//               columns, one weight block), one row per thread
+//               columns, one weight block), one row per thread; at the end of
+//               a tile it writes its 32 x 128 bf16 outputs through a 2 KB
+//               shared-memory buffer with TMA stores
 // Tiles are visited M-fastest so the pairs running at one time share weight
 // tiles through L2. Rows past M and columns past N are zero-filled by TMA
-// and never stored. With per-row weight scales (one per weight row, the
+// and never stored (the output map clips them). With per-row weight scales (one per weight row, the
 // scale block 1 x K of `dequant_fp8_bf16_into`'s per-row layout) the
 // promotion folds in a_s[t][g] only and the epilogue multiplies each output
 // column by its row's scale once.
