@@ -328,3 +328,16 @@ def test_cpu_baseline_sample_sizing():
     calls.clear()
     rows, t = bench.grow_sample(fake(1.0), 1168, 16, 10.0)      # the probe alone exceeds the target
     assert rows == 16 and calls == [16]
+
+
+def test_kernel_digest_ignores_comments_only():
+    """bench.strip_comments: the traffic records stay keyed to a kernel's code,
+    not to its comments; any code change moves the digest."""
+    import bench
+
+    code = "int f(int a) {\n  return a + 1;  // one more\n}\n/* block\n comment */ int g;\n"
+    assert bench.strip_comments(code) == "int f(int a) { return a + 1; } int g;"
+    assert bench.strip_comments(code.replace("one more", "add one")) == bench.strip_comments(code)
+    assert bench.strip_comments(code.replace("a + 1", "a + 2")) != bench.strip_comments(code)
+    for kernel in bench.KERNEL_SOURCES:
+        assert len(bench.kernel_digest(kernel)) == 16
