@@ -212,10 +212,16 @@ struct Cfg {
     static_assert(kSfbCol + 4 * kNBlk * kKSteps <= kTmemCols, "scale columns exceed the allocation");
 };
 
+// Output staging: per epilogue warp, one 32-row x 32-column bf16 block
+// (64-byte rows, 64-byte swizzle) that a TMA store writes to y.
+constexpr uint32_t kOutCols = 32;
+constexpr uint32_t kOutStageBytes = 32 * kOutCols * 2;
+
 template <uint32_t BN, uint32_t AR>
 struct __align__(1024) Smem {
     uint8_t a[Cfg<BN, AR>::kStages][AR * kStageKBytes];
     uint8_t b[Cfg<BN, AR>::kStages][BN * kStageKBytes];
+    uint8_t out[kEpiWarps][kOutStageBytes];
     uint8_t sfa[Cfg<BN, AR>::kStages][kSfStageBytes];
     uint8_t sfb[Cfg<BN, AR>::kStages][Cfg<BN, AR>::kSfbBytes];
     uint64_t full[Cfg<BN, AR>::kStages];
@@ -232,6 +238,8 @@ template <uint32_t BN, uint32_t AR>
 constexpr size_t smem_bytes() {
     return sizeof(Smem<BN, AR>) + 1024;  // + alignment slack
 }
+static_assert(smem_bytes<256, 128>() <= 227 * 1024 && smem_bytes<128, 128>() <= 227 * 1024,
+              "shared memory exceeds the per-CTA limit");
 
 struct Shape {
     uint32_t M, N, K;
@@ -251,8 +259,8 @@ constexpr uint32_t kRedStride = 132;  // floats per partial row (128 + 4: 16-byt
 template <uint32_t BN, uint32_t AR>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb, uint16_t* __restrict__ y,
-                      const Shape sh) {
+                      const __grid_constant__ CUtensorMap tmY, const uint8_t* __restrict__ sfa,
+                      const uint8_t* __restrict__ sfb, uint16_t* __restrict__ y, const Shape sh) {
     using C = Cfg<BN, AR>;
     extern __shared__ uint8_t smem_raw[];
     Smem<BN, AR>& sm =
@@ -289,6 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmY);
     }
     if (warp == 1) {
         tmem_alloc(&sm.tmem_base, C::kTmemCols);
@@ -409,31 +418,54 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 continue;
             }
+            // The warp's 32 rows leave as 32 x 32 bf16 blocks through a 2 KB
+            // shared-memory buffer (16-byte chunk j of row r at chunk
+            // j ^ ((r >> 1) & 3), the 64-byte swizzle of the output map),
+            // stored by one lane with TMA; rows past M are clipped by the map.
+            // The accumulator is released as soon as its last columns are in
+            // registers.
+            const bool rows_live = m0 + quarter * 32u < sh.M;
+            uint8_t* stg = sm.out[warp - 2u];
+            const int32_t y_row = static_cast<int32_t>(m0 + quarter * 32u);
 #pragma unroll 1
             for (uint32_t c = 0; c < BN / 64; ++c) {
                 uint32_t v[64];
                 tmem_load64(tmem + lane_off + buf * BN + c * 64u, v);
-                if (row < sh.M) {
-                    uint4* dst = reinterpret_cast<uint4*>(y + static_cast<size_t>(row) * sh.N + n0 + c * 64u);
+                if (c == BN / 64 - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.acc_empty[buf]);
+                }
+                if (!rows_live) continue;
 #pragma unroll
-                    for (uint32_t j = 0; j < 8; ++j) {
+                for (uint32_t h2 = 0; h2 < 2; ++h2) {
+                    if (lane == 0) bulk_store_wait_read();  // the block before has left the buffer
+                    __syncwarp();
+#pragma unroll
+                    for (uint32_t j = 0; j < 4; ++j) {
                         uint32_t w[4];
 #pragma unroll
                         for (uint32_t h = 0; h < 4; ++h) {
-                            const __nv_bfloat16 e0 = __float2bfloat16_rn(sh.alpha * __uint_as_float(v[8 * j + 2 * h]));
-                            const __nv_bfloat16 e1 =
-                                __float2bfloat16_rn(sh.alpha * __uint_as_float(v[8 * j + 2 * h + 1]));
+                            const uint32_t e = 32 * h2 + 8 * j + 2 * h;
+                            const __nv_bfloat16 e0 = __float2bfloat16_rn(sh.alpha * __uint_as_float(v[e]));
+                            const __nv_bfloat16 e1 = __float2bfloat16_rn(sh.alpha * __uint_as_float(v[e + 1]));
                             w[h] = static_cast<uint32_t>(__bfloat16_as_ushort(e0)) |
                                    (static_cast<uint32_t>(__bfloat16_as_ushort(e1)) << 16);
                         }
-                        dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
+                        *reinterpret_cast<uint4*>(stg + lane * 64u + ((j ^ ((lane >> 1) & 3u)) << 4)) =
+                            make_uint4(w[0], w[1], w[2], w[3]);
                     }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0)
+                        tma_store_2d(&tmY, stg, static_cast<int32_t>(n0 + c * 64u + h2 * kOutCols), y_row);
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.acc_empty[buf]);
         }
+        // Every output block of this warp is in global memory before the CTA
+        // (and its staging buffer) goes away.
+        if (lane == 0) bulk_store_wait_all();
+        __syncwarp();
     }
 
     // After a timed-out wait, let the copies this CTA started land (bounded).
@@ -518,6 +550,21 @@ bool make_map_packed(CUtensorMap* map, const void* base, uint64_t inner, uint64_
     return r == CUDA_SUCCESS;
 }
 
+// The bf16 output y [rows, cols] written in [32 x 32] blocks with the
+// 64-byte swizzle (the GEMM epilogue's staging layout).
+bool make_map_out_bf16(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {kOutCols, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 struct Setup {
     cudaError_t err = cudaSuccess;
     int sms = 0;
@@ -556,8 +603,9 @@ unsigned grid_for(uint64_t items, int sms) {
 
 template <uint32_t BN, uint32_t AR>
 cudaError_t launch_gemm_bn(const Nvfp4GemmLaunch& L, int sms, cudaStream_t stream) {
-    CUtensorMap ta, tb;
-    if (!make_map_packed(&ta, L.qa, L.k / 2, L.m, AR) || !make_map_packed(&tb, L.qw, L.k / 2, L.n, BN))
+    CUtensorMap ta, tb, ty;
+    if (!make_map_packed(&ta, L.qa, L.k / 2, L.m, AR) || !make_map_packed(&tb, L.qw, L.k / 2, L.n, BN) ||
+        !make_map_out_bf16(&ty, L.y, L.n, L.m))
         return cudaErrorInvalidValue;
     Shape sh;
     sh.M = L.m;
@@ -617,7 +665,7 @@ cudaError_t launch_gemm_bn(const Nvfp4GemmLaunch& L, int sms, cudaStream_t strea
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<BN, AR>, ta, tb, static_cast<const uint8_t*>(L.sfa),
+    cudaError_t e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<BN, AR>, ta, tb, ty, static_cast<const uint8_t*>(L.sfa),
                                        static_cast<const uint8_t*>(L.sfw), static_cast<uint16_t*>(L.y), sh);
     note_launch();
     return e != cudaSuccess ? e : cudaGetLastError();
