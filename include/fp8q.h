@@ -423,6 +423,21 @@ fp8q_status fp8q_dequant_fp8_bf16(const void *wq, const float *w_scale, int32_t 
 /* ------------------------------------------------------- diagnostics ---- */
 
 /*
+ * Environment overrides, read once per process, for sweeps:
+ *   FP8Q_QUANT_VARIANT=single|multi  the activation quantizer's variant (the
+ *                                    bytes are the same either way)
+ *   FP8Q_DECODE_SPLIT=<n>            K split of the FP8 GEMM at m <= 64
+ *                                    (CTAs per cluster, at most 8 and k/128)
+ *   FP8Q_NVFP4_SPLIT=<n>             K split of the NVFP4 GEMM when one row of
+ *                                    128-column tiles is used (at most 8 and
+ *                                    k/256)
+ *   FP8Q_LOG=1                       one line on stderr the first time each
+ *                                    quantizer choice is taken
+ * The two splits group the fp32 partial sums differently, so y can change in
+ * its last bits with them; a given split always gives the same y.
+ */
+
+/*
  * Convert `count` fp32 values to E2M1 codes (one per byte, low nibble) with
  * the conversion fp8q_nvfp4_quant uses (round-to-nearest-even, saturating
  * at 6). Used to check the conversion exhaustively. Device pointers.
